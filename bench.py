@@ -1,0 +1,515 @@
+#!/usr/bin/env python
+"""QAM-W codec benchmark: encode/decode Gweights/s of one weight matrix per step.
+
+A *step* is one pass of the whole hot path over one matrix: qamw_calibrate_sigma
+(sigma_k), qamw_encode (channel scale, row norms, rotation, nearest-centroid
+search, packing) and qamw_decode (bf16 weights), all through the C ABI of
+libqamw.so. The default workload is the Llama-7B-shaped attention projection:
+bf16 4096 x 4096, N(0, 0.02^2) with 0.5% outlier columns x20, act RMS
+lognormal(0, 1), alpha 0.5, Hadamard block 128, 2048 centroids (11 bits per
+pair). Inputs are synthetic (seeded); the codebook is the shipped Lloyd table.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...   (one replica per GPU)
+
+Timing: inputs resident in HBM; L2 flushed (256 MiB write) before every timed
+step; CUDA events on the launching stream around each C-ABI call; max over
+ranks. Each rank codes its own matrix (independent problems, no collective on
+the data path), so scaling is weak. ``--impl reference`` times the CPU oracle
+(fp64 numpy) on bounded row samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QAM-W encode/decode Gweights/s per matrix; decode % HBM roofline, encode % FP32"
+FALLBACK_HBM_GBS = 6650.0
+SM_COUNT_B200 = 148
+FP32_LANES_PER_SM = 128
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="llama7b_attn", choices=("llama7b_attn", "tiny", "decode_13b"))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
+    return p.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def workload_spec(name):
+    import synth
+    return synth.WORKLOADS[name]().specs[0], synth.WORKLOADS[name]().name
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm", "clocks.max.sm", "clocks_event_reasons.active", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# multi-rank helpers (also exercised by the gloo tests on CPU)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, seconds_max: float, world: int) -> float:
+    """Whole-job rate: units all ranks processed / the slowest rank's time."""
+    return units_per_rank * world / seconds_max
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(W32_rows, act, spec, C):
+    """calibrate + encode + decode of a row sample with the oracle (fp64 numpy)."""
+    from oracle import codec
+    sig = codec.calibrate_sigma(W32_rows, act, spec.alpha, spec.block, spec.seed)
+    enc = codec.encode(W32_rows, act, spec.alpha, spec.block, spec.seed, sig, C, spec.bits)
+    codec.decode(enc["packed"], enc["r"], sig, act, spec.alpha, spec.K, spec.block, spec.seed, C, spec.bits)
+
+
+def time_oracle(W32, act, spec, C, rows, repeats):
+    from threadpoolctl import threadpool_limits
+    sample = W32[:rows]
+    times = []
+    with threadpool_limits(limits=1):
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            oracle_sample_step(sample, act, spec, C)
+            times.append(time.perf_counter() - t0)
+    return times
+
+
+def auto_rows(spec):
+    """Rows per oracle sample: ~4 s of single-core fp64 work (64 rows of the
+    4096-column, N = 2048 workload; the brute-force search dominates)."""
+    per_row = spec.K / 2 * spec.N
+    return max(1, min(spec.M, int(round(64 * 2048 * 2048 / per_row))))
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import synth
+    import vector_codebook_codec_b200 as q
+    spec, wname = workload_spec(args.workload)
+    W32 = synth.make_matrix(spec)
+    if spec.dtype == "bf16":
+        _, W32 = synth.to_bf16(W32)
+    act = synth.act_for(spec)
+    C = q.load_codebook(spec.N)
+    rows = args.cpu_rows or auto_rows(spec)
+    for _ in range(args.warmup):
+        time_oracle(W32, act, spec, C, rows, 1)
+    times = time_oracle(W32, act, spec, C, rows, args.steps)
+    tot = sum(times)
+    value = rows * spec.K * args.steps / tot / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wname, "M": spec.M, "K": spec.K, "block": spec.block, "N": spec.N,
+                   "bits": spec.bits, "alpha": spec.alpha, "weight_dtype": spec.dtype},
+        "cpu_baseline": {"value": value, "unit": "Gweights/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {rows} of {spec.M} rows per step (calibrate + encode + decode)"},
+        "e2e": {"value": value, "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_decode_sweep(args):
+    """Decode-only steps over the 13B-shaped matrices (5120x5120, 13824x5120,
+    5120x13824), pre-encoded on the GPU outside the timed region; one step
+    decodes all three to bf16."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import vector_codebook_codec_b200 as q
+    from vector_codebook_codec_b200 import build as qbuild
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    qbuild.build()
+    wl = synth.decode_sweep_13b()
+    mats = []
+    for spec in wl.specs:
+        Wt, _ = synth.to_bf16(synth.make_matrix(spec))
+        Wd = Wt.to(dev)
+        act = torch.from_numpy(synth.act_for(spec)).to(dev)
+        Cd = torch.from_numpy(q.load_codebook(spec.N)).to(dev)
+        sig = q.calibrate_sigma(Wd, act, spec.alpha, spec.block, spec.seed)
+        enc = q.encode(Wd, act, spec.alpha, spec.block, spec.seed, sig, Cd, spec.bits)
+        del Wd
+        out = torch.empty((spec.M, spec.K), dtype=torch.bfloat16, device=dev)
+        mats.append((spec, enc, Cd, out))
+    torch.cuda.synchronize(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nm = len(mats)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nm + 1)] for _ in range(args.steps)]
+
+    def one(evs=None):
+        for j, (spec, enc, Cd, out) in enumerate(mats):
+            if evs: evs[j].record(stream)
+            q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=out)
+        if evs: evs[nm].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        one(ev[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()}")
+    per = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j in range(nm)]
+    total_s = max_over_ranks(sum(ev[i][0].elapsed_time(ev[i][nm]) for i in range(args.steps)) / 1e3, dev)
+    weights = sum(sp.M * sp.K for sp, _, _, _ in mats)
+    value = aggregate_throughput(weights * args.steps, total_s, world) / 1e9
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    per_mat = []
+    tot_bytes = 0
+    for (spec, enc, _, _), t in zip(mats, per):
+        wpr = q.words_per_row(spec.K, spec.bits)
+        b = spec.M * spec.K * 2 + spec.M * wpr * 4 + 4 * spec.M + 4 * spec.K + 2 * spec.K + 8 * spec.N
+        tot_bytes += b
+        ms = statistics.mean(t)
+        per_mat.append({"name": spec.name, "M": spec.M, "K": spec.K, "us": 1e3 * ms,
+                        "gweights_per_s": spec.M * spec.K / (ms * 1e-3) / 1e9,
+                        "gbs": b / (ms * 1e-3) / 1e9, "frac": b / (ms * 1e-3) / 1e9 / hbm})
+    mean_step_s = total_s / args.steps
+    roof = {"bound": "hbm", "achieved": tot_bytes / mean_step_s / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": tot_bytes / mean_step_s / 1e9 / hbm, "traffic": None, "kernel": "decode_kernel",
+            "peak_source": f"{peak_kind} hbm_gbs"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * mean_step_s, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no checkpoint)",
+                "config": {"workload": wl.name, "op": "decode only (bf16 out)", "matrices": [
+                    f"{sp.M}x{sp.K}" for sp, _, _, _ in mats], "block": 128, "N": 2048, "bits": 11,
+                    "l2": "flushed by a 256 MiB write before every timed step",
+                    "parallelism": f"{world} independent replica(s)"},
+                "roofline": roof, "per_matrix": per_mat, "gpu_launches": nm * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_ours(args):
+    if args.workload == "decode_13b":
+        return run_decode_sweep(args)
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import vector_codebook_codec_b200 as q
+    from vector_codebook_codec_b200 import build as qbuild
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    qbuild.build()
+    q.load_library()
+
+    spec, wname = workload_spec(args.workload)
+    M, K = spec.M, spec.K
+    w32 = synth.make_matrix(spec)
+    if spec.dtype == "bf16":
+        Wt, W32 = synth.to_bf16(w32)
+    else:
+        import torch as _t
+        Wt, W32 = _t.from_numpy(w32), w32
+    act = synth.act_for(spec)
+    C = q.load_codebook(spec.N)
+    Wd = Wt.to(dev)
+    actd = torch.from_numpy(act).to(dev)
+    Cd = torch.from_numpy(C).to(dev)
+    lib = q.load_library()
+    wpr = q.words_per_row(K, spec.bits)
+    ws = torch.empty(int(lib.qamw_calibrate_workspace_bytes(M, K)), dtype=torch.uint8, device=dev)
+    sigma = torch.empty(K // 2, dtype=torch.float32, device=dev)
+    packed = torch.empty((M, wpr), dtype=torch.int32, device=dev)
+    rnorm = torch.empty(M, dtype=torch.float32, device=dev)
+    cscale = torch.empty(K, dtype=torch.float32, device=dev)
+    out = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(max(args.steps, 1))]
+
+    def one(evs=None):
+        if evs: evs[0].record(stream)
+        sig = q.calibrate_sigma(Wd, actd, spec.alpha, spec.block, spec.seed, status=status, workspace=ws,
+                                out=sigma)
+        if evs: evs[1].record(stream)
+        enc = q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sig, Cd, spec.bits, status=status,
+                       out=(packed, rnorm, cscale))
+        if evs: evs[2].record(stream)
+        q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=out)
+        if evs: evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()} after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        one(ev[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    clk = clocks.stop()
+
+    t_cal = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    t_enc = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    t_dec = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    t_step = [ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    total_s = max_over_ranks(sum(t_step) / 1e3, dev)
+    weights = M * K
+    value = aggregate_throughput(weights * args.steps, total_s, world) / 1e9
+
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    fp32_peak = sms * FP32_LANES_PER_SM * sm_max * 1e6  # FP32 lane-instructions per second
+    P = M * K // 2
+    enc_ops = 4.0 * P * spec.N              # 2 sub + 1 mul + 1 fma per (pair, centroid)
+    enc_ms = statistics.mean(t_enc)
+    dec_ms = statistics.mean(t_dec)
+    cal_ms = statistics.mean(t_cal)
+    dec_bytes = M * K * 2 + M * wpr * 4 + 4 * M + 4 * K + 2 * K + 8 * spec.N
+    cal_bytes = M * K * 2 * 2 + 4 * K + 4 * M
+    enc_roof = {"bound": "alu", "achieved": enc_ops / (enc_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
+                "unit": "Gop/s", "frac": enc_ops / (enc_ms * 1e-3) / fp32_peak, "traffic": None,
+                "kernel": "encode_kernel (brute-force search; events span the qamw_encode call)",
+                "peak_source": f"{sms} SMs x 128 FP32 lanes x {sm_max:.0f} MHz ({peak_kind} max clock)"}
+    dec_roof = {"bound": "hbm", "achieved": dec_bytes / (dec_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": dec_bytes / (dec_ms * 1e-3) / 1e9 / hbm, "traffic": None, "kernel": "decode_kernel",
+                "peak_source": f"{peak_kind} hbm_gbs", "gweights_per_s": weights / (dec_ms * 1e-3) / 1e9}
+    cal_roof = {"bound": "hbm", "achieved": cal_bytes / (cal_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": cal_bytes / (cal_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+                "kernel": "qamw_calibrate_sigma (4 kernels)"}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Wh = Wt.pin_memory()
+        acth = torch.from_numpy(act).pin_memory()
+        outh = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+        pkh = torch.empty((M, wpr), dtype=torch.int32).pin_memory()
+        rh = torch.empty(M, dtype=torch.float32).pin_memory()
+        sh = torch.empty(K, dtype=torch.float32).pin_memory()
+        sgh = torch.empty(K // 2, dtype=torch.float32).pin_memory()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            Wd.copy_(Wh, non_blocking=True)
+            actd.copy_(acth, non_blocking=True)
+            one()
+            outh.copy_(out, non_blocking=True)
+            pkh.copy_(packed, non_blocking=True)
+            rh.copy_(rnorm, non_blocking=True)
+            sh.copy_(cscale, non_blocking=True)
+            sgh.copy_(sigma, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+        e2e = {"value": aggregate_throughput(weights * args.steps, e2e_s, world) / 1e9, "unit": "Gweights/s",
+               "h2d_bytes_per_step": Wh.numel() * 2 + acth.numel() * 4,
+               "d2h_bytes_per_step": outh.numel() * 2 + pkh.numel() * 4 + 4 * M + 4 * K + 2 * K}
+
+    # ---- oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = args.cpu_rows or auto_rows(spec)
+        times = time_oracle(W32, act, spec, C, rows, 3)
+        cpu = {"value": rows * K / statistics.median(times) / 1e9, "unit": "Gweights/s", "cores": 1,
+               "kind": "oracle",
+               "sample": f"{rows} of {M} rows, calibrate + encode + decode, median of 3 (fp64 numpy, 1 thread)"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; no checkpoint)",
+            "config": {"workload": wname, "M": M, "K": K, "weight_dtype": spec.dtype, "block": spec.block,
+                       "N": spec.N, "bits": spec.bits, "alpha": spec.alpha, "search": "brute-force",
+                       "l2": "flushed by a 256 MiB write before every timed step",
+                       "parallelism": f"{world} independent replica(s)"},
+            "roofline": enc_roof,
+            "rooflines": {"encode": enc_roof, "decode": dec_roof, "calibrate": cal_roof},
+            "ms": {"calibrate": cal_ms, "encode": enc_ms, "decode": dec_ms},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 8 * args.steps, "clocks": clk,
+            "dtype_detail": "rotation fp64, search and decode fp32, decode output bf16",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,179 @@
+/*
+ * qamw.h -- C ABI of libqamw.so, the sm_100a (B200) QAM-W weight codec.
+ *
+ * The method: "QAM-W: Joint 2D Codebook Quantization for LLM Weights via
+ * Hadamard Rotation and Activation-Aware Scaling" (gist.science/paper/2605.26339),
+ * Technical Summary, "Methodology: The QAM-W Codec", steps
+ *   (1) Separation of Scale and Direction  (2) Deterministic Rotation
+ *   (3) Pairing and Calibration            (4) Joint 2D Quantization
+ *   (5) Activation-Aware Scaling           (6) Decoding.
+ * Step (5) is applied before quantization, so a row is coded as
+ *   w'_j = w_j * s_j                     s_j = RN32(act_rms_j ^ alpha), pow in fp64   (5)
+ *   r    = RN32(||w'||_2)                stored row norm                               (1)
+ *   y    = H_b (d * w'/r) / sqrt(b)      per block of b columns, d_j = +-1 mask         (2)
+ *   z_k  = (y_2k, y_2k+1),  x_k = RN32(z_k / sigma_k)                                  (3)
+ *   idx_k = argmin_c |x_k - C_c|^2       lowest index on ties                          (4)
+ * and decoded as w_hat = r * d * (H_b (sigma (.) C[idx])) / (sqrt(b) * s)           (6).
+ * H_b is the Sylvester (natural order) Hadamard matrix; d_j = -1 exactly when
+ * bit 63 of the (j+1)-th SplitMix64 output for sign_seed is set (one mask per
+ * matrix, shared by all rows).
+ *
+ * Conventions shared by every entry point
+ *   - Every array pointer is a DEVICE pointer owned by the caller; the library
+ *     keeps no allocation and no global state between calls.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return once the kernels are enqueued.
+ *   - Arguments are validated on the host before anything is launched; on a
+ *     validation error nothing is enqueued and the status code says why.
+ *   - Shapes: W is M x K, row-major with leading dimension ld >= K (elements).
+ *     K must be even and a multiple of the block size b; b is a power of two
+ *     in [2, 1024]; 1 <= bits_per_pair <= 16; 1 <= N <= min(2^bits, 8192).
+ *   - Packed index stream: uint32 [M][qamw_words_per_row(K, bits)], each row
+ *     starting on a fresh word; index k of a row occupies stream bits
+ *     k*bits .. k*bits+bits-1, least significant bit first, and stream bit t is
+ *     bit (t mod 32) of word t/32 (little-endian words).
+ *   - Codebook: float32 [N][2] (x, y) centroids, row-major.
+ *   - `status` (nullable) is a device int32 the kernels OR bits into
+ *     (QAMW_STATUS_*); the caller clears it and reads it after syncing.
+ *   - Return value: QAMW_OK or an error code below; qamw_last_error() gives a
+ *     message for the most recent failing call on the calling host thread.
+ */
+#ifndef QAMW_H_
+#define QAMW_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qamw_stream_t; /* same type as cudaStream_t */
+
+typedef enum { QAMW_F32 = 0, QAMW_BF16 = 1 } qamw_dtype;
+
+/* Return codes. */
+enum {
+  QAMW_OK = 0,
+  QAMW_EINVAL = 1,       /* bad shape or argument value */
+  QAMW_ENULL = 2,        /* a required pointer is NULL */
+  QAMW_EUNSUPPORTED = 3, /* valid for the method but beyond this build's limits */
+  QAMW_ECUDA = 4,        /* a CUDA call failed (see qamw_last_error) */
+  QAMW_EWORKSPACE = 5    /* workspace missing or smaller than required */
+};
+
+/* Device status bits (ORed into *status by the kernels). */
+#define QAMW_STATUS_BAD_INDEX 1u        /* decode: an index >= N (decoded as 0) */
+#define QAMW_STATUS_NONFINITE_NORM 2u   /* a row norm is Inf/NaN */
+#define QAMW_STATUS_BAD_ACT_RMS 4u      /* an act_rms entry is not finite and > 0 */
+#define QAMW_STATUS_NONFINITE_INPUT 8u  /* a weight is Inf/NaN (its pairs coded as index 0) */
+#define QAMW_STATUS_TIMEOUT 16u         /* a bounded wait on an asynchronous copy ran out; output incomplete */
+
+/* Maximum sizes of this build. */
+#define QAMW_MAX_CENTROIDS 8192
+#define QAMW_MAX_BLOCK 1024
+
+/* Words per row of the packed stream: ceil((K/2) * bits / 32); -1 if invalid. */
+int64_t qamw_words_per_row(int64_t K, int32_t bits_per_pair);
+
+/* Message for a return code (static string). */
+const char *qamw_status_string(int code);
+
+/* Message of the most recent failing call on this host thread ("" if none). */
+const char *qamw_last_error(void);
+
+/* Version string of the library. */
+const char *qamw_version(void);
+
+/*
+ * qamw_channel_scale -- Methodology (5) Activation-Aware Scaling.
+ * s_out[j] = RN32(pow((double)act_rms[j], (double)alpha)) for j < K; the
+ * proportionality constant is 1. act_rms == NULL writes s = 1. Entries that
+ * are not finite and > 0 give s = 1 and set QAMW_STATUS_BAD_ACT_RMS.
+ *   act_rms  : device float32 [K] or NULL      s_out : device float32 [K]
+ */
+int qamw_channel_scale(const float *act_rms, float alpha, int64_t K, float *s_out,
+                       int32_t *status, qamw_stream_t stream);
+
+/*
+ * qamw_calibrate_workspace_bytes -- scratch needed by qamw_calibrate_sigma.
+ */
+size_t qamw_calibrate_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * qamw_calibrate_sigma -- Methodology (3) Pairing and Calibration.
+ * sigma_out[k] = RN32(sqrt(2/pi) * (1/M) * sum_i |z_ik|) for k < K/2, the
+ * Rayleigh mean-amplitude estimate that maps pair k onto the unit circular
+ * Gaussian; a pair position that is zero in every row gets 1.0. z is computed
+ * exactly as in qamw_encode (steps 5, 1, 2). The sum runs in fp64 over fixed
+ * row groups and is reduced in a fixed order, so the result is deterministic.
+ *   W        : device [M][ldw] of w_dtype        act_rms : device float32 [K] or NULL (s = 1)
+ *   sigma_out: device float32 [K/2]              workspace: device, >= qamw_calibrate_workspace_bytes(M, K)
+ * Errors: QAMW_ENULL (W, sigma_out, workspace), QAMW_EINVAL (shape, alpha not
+ * finite, M < 1), QAMW_EWORKSPACE.
+ */
+int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                         const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                         float *sigma_out, void *workspace, size_t workspace_bytes,
+                         int32_t *status, qamw_stream_t stream);
+
+/*
+ * qamw_encode -- Methodology steps (5), (1), (2), (3), (4) and bit packing.
+ * For every row: s_j (step 5), r_i = RN32(||w' ||) written to row_norm_out
+ * (step 1), the sign-masked block Hadamard rotation (step 2, in fp64, so that
+ * x_k = RN32(z_k / sigma_k) is the correctly rounded value), pairing with the
+ * given sigma (step 3), the nearest centroid by fp32 direct-difference squared
+ * distance (x0-c0)^2 + (x1-c1)^2 with the lowest index on ties (step 4), and
+ * the packed stream described above. A zero row codes x = 0.
+ *   W           : device [M][ldw] of w_dtype       act_rms : device float32 [K] or NULL
+ *   sigma       : device float32 [K/2] (from qamw_calibrate_sigma, all > 0)
+ *   codebook    : device float32 [N][2]
+ *   search_table: device table from qamw_build_search_table for this codebook,
+ *                 or NULL for the brute-force search over all N centroids.
+ *                 Both searches return the same index.
+ *   packed_out  : device uint32 [M][qamw_words_per_row(K, bits)]
+ *   row_norm_out: device float32 [M]                 col_scale_out: device float32 [K] (s_j)
+ * row_norm_out and col_scale_out are the metadata qamw_decode needs; the
+ * encode also reads them back between its kernels (no other scratch).
+ * Errors: QAMW_ENULL, QAMW_EINVAL (shape, code size, alpha), QAMW_EUNSUPPORTED.
+ */
+int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                const float *sigma, const float *codebook, int32_t N, int32_t bits_per_pair,
+                const void *search_table, uint32_t *packed_out, float *row_norm_out,
+                float *col_scale_out, int32_t *status, qamw_stream_t stream);
+
+/*
+ * qamw_decode -- Methodology (6) Decoding.
+ * w_hat_ij = r_i * d_j * (H_b (sigma (.) C[idx]))_j / (sqrt(b) * s_j): unpack,
+ * look up centroids, rescale by sigma_k, inverse rotation, multiply by the
+ * stored row norm, divide by the stored channel scale. fp32 arithmetic; the
+ * output is rounded (RNE) to out_dtype. bf16 output is what the page's pipeline
+ * feeds to the matrix multiply ("Significance and Claims").
+ *   packed   : device uint32 [M][qamw_words_per_row(K, bits)]
+ *   row_norm : device float32 [M]      sigma : device float32 [K/2]
+ *   col_scale: device float32 [K] (s_j as written by qamw_encode) or NULL (s = 1)
+ *   codebook : device float32 [N][2]   W_out : device [M][ldo] of out_dtype
+ * An index >= N decodes as centroid 0 and sets QAMW_STATUS_BAD_INDEX; a
+ * non-finite row norm sets QAMW_STATUS_NONFINITE_NORM.
+ */
+int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigma,
+                const float *col_scale, int64_t M, int64_t K, int32_t block,
+                uint64_t sign_seed, const float *codebook, int32_t N, int32_t bits_per_pair,
+                void *W_out, qamw_dtype out_dtype, int64_t ldo, int32_t *status,
+                qamw_stream_t stream);
+
+/*
+ * qamw_rotate_rows -- the rotation alone, for tests of step (2).
+ * inverse == 0: Y = H_b (d * U) / sqrt(b); inverse != 0: Y = d * (H_b U) / sqrt(b),
+ * per block of b columns, in fp64 (the encode path's arithmetic).
+ *   U, Y : device float64 [M][K] (dense, ld = K)
+ */
+int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t block,
+                     uint64_t sign_seed, int32_t inverse, qamw_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QAMW_H_ */

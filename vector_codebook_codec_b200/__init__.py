@@ -1,0 +1,263 @@
+"""vector_codebook_codec_b200 -- Python binding of libqamw.so, the sm_100a QAM-W codec.
+
+The library implements the row-parallel encode and decode of QAM-W ("QAM-W:
+Joint 2D Codebook Quantization for LLM Weights via Hadamard Rotation and
+Activation-Aware Scaling", Technical Summary, "Methodology: The QAM-W Codec").
+Every step of the codec runs in the CUDA kernels of ``libqamw.so``; this module
+only marshals arguments: it checks tensor devices, dtypes and shapes, passes raw
+device pointers and the current CUDA stream through the C ABI declared in
+``include/qamw.h``, and raises on a non-zero status. PyTorch provides device
+memory and streams only. There is no CPU fallback: if the library is missing
+or was built for another GPU the calls raise.
+
+Functions with the C names (``qamw_calibrate_sigma``, ``qamw_encode``,
+``qamw_decode``, ...) take raw pointers exactly like the C ABI; the
+lower-case helpers (``calibrate_sigma``, ``encode``, ``decode``) take torch
+tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqamw.so")
+CODEBOOK_DIR = os.path.join(_PKG, "codebooks")
+
+QAMW_F32, QAMW_BF16 = 0, 1
+QAMW_OK, QAMW_EINVAL, QAMW_ENULL, QAMW_EUNSUPPORTED, QAMW_ECUDA, QAMW_EWORKSPACE = range(6)
+STATUS_BAD_INDEX, STATUS_NONFINITE_NORM, STATUS_BAD_ACT_RMS, STATUS_NONFINITE_INPUT, STATUS_TIMEOUT = 1, 2, 4, 8, 16
+
+_c_i64, _c_i32, _c_u64, _c_f32, _c_sz, _c_p = (ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64,
+                                               ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p)
+
+# name -> (restype, argtypes); mirrors include/qamw.h
+_SIGNATURES = {
+    "qamw_words_per_row": (_c_i64, [_c_i64, _c_i32]),
+    "qamw_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qamw_last_error": (ctypes.c_char_p, []),
+    "qamw_version": (ctypes.c_char_p, []),
+    "qamw_channel_scale": (ctypes.c_int, [_c_p, _c_f32, _c_i64, _c_p, _c_p, _c_p]),
+    "qamw_calibrate_workspace_bytes": (_c_sz, [_c_i64, _c_i64]),
+    "qamw_calibrate_sigma": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32,
+                                            _c_u64, _c_p, _c_p, _c_sz, _c_p, _c_p]),
+    "qamw_encode": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32, _c_u64,
+                                   _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    "qamw_decode": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
+                                   _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
+    "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
+}
+
+_lib = None
+
+
+class QamwError(RuntimeError):
+    """A libqamw call returned a non-zero status."""
+
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libqamw.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libqamw.so not found at {path}; build it with "
+                          f"`python -m vector_codebook_codec_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, rc: int):
+    if rc != QAMW_OK:
+        lib = load_library()
+        raise QamwError(fn, rc, lib.qamw_last_error().decode() or lib.qamw_status_string(rc).decode())
+
+
+def _raw(name):
+    def call(*args):
+        return getattr(load_library(), name)(*args)
+    call.__name__ = name
+    call.__doc__ = f"Raw C-ABI call {name} (see include/qamw.h)."
+    return call
+
+
+# Raw C-ABI entry points under their C names.
+qamw_words_per_row = _raw("qamw_words_per_row")
+qamw_status_string = _raw("qamw_status_string")
+qamw_last_error = _raw("qamw_last_error")
+qamw_version = _raw("qamw_version")
+qamw_channel_scale = _raw("qamw_channel_scale")
+qamw_calibrate_workspace_bytes = _raw("qamw_calibrate_workspace_bytes")
+qamw_calibrate_sigma = _raw("qamw_calibrate_sigma")
+qamw_encode = _raw("qamw_encode")
+qamw_decode = _raw("qamw_decode")
+qamw_rotate_rows = _raw("qamw_rotate_rows")
+
+
+# ---------------------------------------------------------------------------
+# torch-tensor helpers (argument marshalling only)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D")
+
+
+def _wdtype(W):
+    torch = _torch()
+    if W.dtype == torch.bfloat16:
+        return QAMW_BF16
+    if W.dtype == torch.float32:
+        return QAMW_F32
+    raise ValueError("W must be bfloat16 or float32")
+
+
+def _ld(W):
+    if W.stride(1) != 1:
+        raise ValueError("W must be row-major with unit column stride")
+    return W.stride(0) if W.shape[0] > 1 else W.shape[1]
+
+
+def words_per_row(K: int, bits: int) -> int:
+    return int(load_library().qamw_words_per_row(K, bits))
+
+
+def load_codebook(N: int):
+    """The shipped joint 2D Lloyd-Max codebook with N centroids (float32 numpy [N, 2])."""
+    path = os.path.join(CODEBOOK_DIR, f"qamw_lloyd_N{N}.npy")
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"no shipped codebook with N={N} ({path})")
+    return np.load(path).astype(np.float32)
+
+
+def codebook_manifest() -> dict:
+    with open(os.path.join(CODEBOOK_DIR, "manifest.json")) as f:
+        return json.load(f)
+
+
+def channel_scale(act_rms, alpha: float, K: int, status=None, stream=None):
+    torch = _torch()
+    _need_cuda("act_rms", act_rms, torch.float32, 1)
+    s = torch.empty(K, dtype=torch.float32, device="cuda" if act_rms is None else act_rms.device)
+    _check("qamw_channel_scale", load_library().qamw_channel_scale(
+        _ptr(act_rms), float(alpha), K, _ptr(s), _ptr(status), _stream_ptr(stream)))
+    return s
+
+
+def calibrate_sigma(W, act_rms, alpha: float, block: int, seed: int, status=None, workspace=None,
+                    stream=None, out=None):
+    """sigma_k for every pair position of W (float32 [K/2]); see qamw_calibrate_sigma."""
+    torch = _torch()
+    _need_cuda("W", W, ndim=2)
+    _need_cuda("act_rms", act_rms, torch.float32, 1)
+    M, K = W.shape
+    lib = load_library()
+    need = int(lib.qamw_calibrate_workspace_bytes(M, K))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    sigma = torch.empty(K // 2, dtype=torch.float32, device=W.device) if out is None else out
+    _check("qamw_calibrate_sigma", lib.qamw_calibrate_sigma(
+        _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
+        _ptr(sigma), _ptr(workspace), workspace.numel(), _ptr(status), _stream_ptr(stream)))
+    return sigma
+
+
+@dataclass
+class Encoded:
+    """An encoded matrix: the stored artefacts the decode needs."""
+    packed: object      # uint32 stored as torch.int32 [M, words_per_row]
+    row_norm: object    # float32 [M]
+    col_scale: object   # float32 [K]  (s_j)
+    sigma: object       # float32 [K/2]
+    M: int
+    K: int
+    block: int
+    seed: int
+    N: int
+    bits: int
+
+
+def encode(W, act_rms, alpha: float, block: int, seed: int, sigma, codebook, bits: int,
+           status=None, stream=None, out=None) -> Encoded:
+    """Encode W with the given sigma and codebook (float32 CUDA tensor [N, 2])."""
+    torch = _torch()
+    _need_cuda("W", W, ndim=2)
+    _need_cuda("act_rms", act_rms, torch.float32, 1)
+    _need_cuda("sigma", sigma, torch.float32, 1)
+    _need_cuda("codebook", codebook, torch.float32, 2)
+    M, K = W.shape
+    N = codebook.shape[0]
+    wpr = words_per_row(K, bits)
+    if wpr < 0:
+        raise ValueError("invalid K / bits")
+    if out is None:
+        packed = torch.empty((M, wpr), dtype=torch.int32, device=W.device)
+        r = torch.empty(M, dtype=torch.float32, device=W.device)
+        s = torch.empty(K, dtype=torch.float32, device=W.device)
+    else:
+        packed, r, s = out
+    _check("qamw_encode", load_library().qamw_encode(
+        _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
+        _ptr(sigma), _ptr(codebook.contiguous()), N, bits, None, _ptr(packed), _ptr(r), _ptr(s),
+        _ptr(status), _stream_ptr(stream)))
+    return Encoded(packed, r, s, sigma, M, K, block, seed, N, bits)
+
+
+def decode(enc: Encoded, codebook, out_dtype=None, status=None, stream=None, out=None):
+    """Decode an :class:`Encoded` matrix to bf16 (default) or fp32 [M, K]."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    ot = QAMW_BF16 if out_dtype == torch.bfloat16 else QAMW_F32
+    if out is None:
+        out = torch.empty((enc.M, enc.K), dtype=out_dtype, device=enc.packed.device)
+    _check("qamw_decode", load_library().qamw_decode(
+        _ptr(enc.packed), _ptr(enc.row_norm), _ptr(enc.sigma), _ptr(enc.col_scale), enc.M, enc.K,
+        enc.block, enc.seed & (2**64 - 1), _ptr(codebook.contiguous()), codebook.shape[0], enc.bits,
+        _ptr(out), ot, _ld(out), _ptr(status), _stream_ptr(stream)))
+    return out
+
+
+def rotate_rows(U, block: int, seed: int, inverse: bool = False, stream=None):
+    """The rotation alone on float64 rows (test hook of the encode's fp64 rotation)."""
+    torch = _torch()
+    _need_cuda("U", U, torch.float64, 2)
+    U = U.contiguous()
+    Y = torch.empty_like(U)
+    M, K = U.shape
+    _check("qamw_rotate_rows", load_library().qamw_rotate_rows(
+        _ptr(U), _ptr(Y), M, K, block, seed & (2**64 - 1), 1 if inverse else 0, _stream_ptr(stream)))
+    return Y

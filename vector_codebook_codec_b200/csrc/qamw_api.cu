@@ -1,0 +1,246 @@
+// qamw_api.cu -- the extern "C" entry points of libqamw.so (declared in
+// include/qamw.h): host-side argument validation, workspace carving and the
+// kernel launches. Nothing is allocated; nothing is launched when an argument
+// is rejected.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "qamw.h"
+#include "qamw_internal.h"
+
+namespace qamw {
+
+namespace {
+thread_local char g_last_error[512] = {0};
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where) {
+  return fail(QAMW_ECUDA, "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int log2i(int64_t v) {
+  int l = 0;
+  while ((int64_t(1) << l) < v) ++l;
+  return l;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Shape checks common to calibrate / encode / decode.
+int check_shape(int64_t M, int64_t K, int32_t block, const char *fn) {
+  if (M < 1) return fail(QAMW_EINVAL, "%s: M must be >= 1 (got %lld)", fn, (long long)M);
+  if (K < 2 || (K & 1)) return fail(QAMW_EINVAL, "%s: K must be even and >= 2 (got %lld)", fn, (long long)K);
+  if (!is_pow2(block) || block < 2)
+    return fail(QAMW_EINVAL, "%s: block must be a power of two >= 2 (got %d)", fn, block);
+  if (block > QAMW_MAX_BLOCK)
+    return fail(QAMW_EUNSUPPORTED, "%s: block %d exceeds %d", fn, block, QAMW_MAX_BLOCK);
+  if (K % block) return fail(QAMW_EINVAL, "%s: K (%lld) must be a multiple of block (%d)", fn, (long long)K, block);
+  if (M > (int64_t(1) << 40) || K > (int64_t(1) << 31))
+    return fail(QAMW_EUNSUPPORTED, "%s: shape too large", fn);
+  return QAMW_OK;
+}
+
+int check_code(int32_t N, int32_t bits, const char *fn) {
+  if (bits < 1 || bits > 16) return fail(QAMW_EINVAL, "%s: bits_per_pair must be in [1, 16] (got %d)", fn, bits);
+  if (N < 1 || (int64_t)N > (int64_t(1) << bits))
+    return fail(QAMW_EINVAL, "%s: need 1 <= N <= 2^bits (N=%d, bits=%d)", fn, N, bits);
+  if (N > QAMW_MAX_CENTROIDS)
+    return fail(QAMW_EUNSUPPORTED, "%s: N=%d exceeds %d centroids", fn, N, QAMW_MAX_CENTROIDS);
+  return QAMW_OK;
+}
+
+int check_dtype(qamw_dtype t, const char *fn) {
+  if (t != QAMW_F32 && t != QAMW_BF16) return fail(QAMW_EINVAL, "%s: unknown dtype %d", fn, (int)t);
+  return QAMW_OK;
+}
+
+std::mutex g_sm_mu;
+int g_sm_count[64] = {0};
+}  // namespace
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(g_sm_mu);
+  if (g_sm_count[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_sm_count[dev] = v;
+  }
+  return g_sm_count[dev];
+}
+
+}  // namespace qamw
+
+using namespace qamw;
+
+extern "C" {
+
+const char *qamw_version(void) { return "qamw 0.1.0 (sm_100a)"; }
+
+const char *qamw_status_string(int code) {
+  switch (code) {
+    case QAMW_OK: return "ok";
+    case QAMW_EINVAL: return "invalid argument";
+    case QAMW_ENULL: return "null pointer";
+    case QAMW_EUNSUPPORTED: return "unsupported by this build";
+    case QAMW_ECUDA: return "CUDA error";
+    case QAMW_EWORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+const char *qamw_last_error(void) { return g_last_error; }
+
+int64_t qamw_words_per_row(int64_t K, int32_t bits_per_pair) {
+  if (K < 2 || (K & 1) || bits_per_pair < 1 || bits_per_pair > 16) return -1;
+  return ((K / 2) * bits_per_pair + 31) / 32;
+}
+
+int qamw_channel_scale(const float *act_rms, float alpha, int64_t K, float *s_out, int32_t *status,
+                       qamw_stream_t stream) {
+  g_last_error[0] = 0;
+  if (s_out == nullptr) return fail(QAMW_ENULL, "qamw_channel_scale: s_out is NULL");
+  if (K < 1) return fail(QAMW_EINVAL, "qamw_channel_scale: K must be >= 1");
+  if (!std::isfinite(alpha)) return fail(QAMW_EINVAL, "qamw_channel_scale: alpha must be finite");
+  ScaleArgs a{act_rms, alpha, K, s_out, status};
+  cudaError_t e = launch_channel_scale(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, "qamw_channel_scale");
+}
+
+size_t qamw_calibrate_workspace_bytes(int64_t M, int64_t K) {
+  if (M < 1 || K < 2) return 0;
+  const int64_t groups = (M + kCalibRowGroup - 1) / kCalibRowGroup;
+  return align256((size_t)K * 4) + align256((size_t)M * 4) + align256((size_t)groups * (size_t)(K / 2) * 8);
+}
+
+int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                         const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                         float *sigma_out, void *workspace, size_t workspace_bytes, int32_t *status,
+                         qamw_stream_t stream) {
+  static const char *fn = "qamw_calibrate_sigma";
+  g_last_error[0] = 0;
+  int rc;
+  if (W == nullptr || sigma_out == nullptr) return fail(QAMW_ENULL, "%s: W and sigma_out must be non-NULL", fn);
+  if ((rc = check_dtype(w_dtype, fn))) return rc;
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
+  if (!std::isfinite(alpha)) return fail(QAMW_EINVAL, "%s: alpha must be finite", fn);
+  const size_t need = qamw_calibrate_workspace_bytes(M, K);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(QAMW_EWORKSPACE, "%s: workspace of %zu bytes needed (got %zu)", fn, need, workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(QAMW_EINVAL, "%s: workspace must be 256-byte aligned", fn);
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  float *s = reinterpret_cast<float *>(ws);
+  float *r = reinterpret_cast<float *>(ws + align256((size_t)K * 4));
+  double *partials = reinterpret_cast<double *>(ws + align256((size_t)K * 4) + align256((size_t)M * 4));
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = launch_channel_scale(ScaleArgs{act_rms, alpha, K, s, status}, st)) != cudaSuccess) return cuda_fail(e, fn);
+  if ((e = launch_row_norms(RowNormArgs{W, w_dtype, M, K, ldw, s, r, status}, st)) != cudaSuccess)
+    return cuda_fail(e, fn);
+  CalibArgs ca;
+  ca.rot = RotateArgs{W, w_dtype, M, K, ldw, log2i(block), sign_seed, s, r};
+  ca.partials = partials;
+  ca.groups = (M + kCalibRowGroup - 1) / kCalibRowGroup;
+  ca.sigma_out = sigma_out;
+  if ((e = launch_calibrate(ca, st)) != cudaSuccess) return cuda_fail(e, fn);
+  return QAMW_OK;
+}
+
+int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                const float *sigma, const float *codebook, int32_t N, int32_t bits_per_pair,
+                const void *search_table, uint32_t *packed_out, float *row_norm_out,
+                float *col_scale_out, int32_t *status, qamw_stream_t stream) {
+  static const char *fn = "qamw_encode";
+  g_last_error[0] = 0;
+  int rc;
+  if (!W || !sigma || !codebook || !packed_out || !row_norm_out || !col_scale_out)
+    return fail(QAMW_ENULL, "%s: W, sigma, codebook, packed_out, row_norm_out, col_scale_out must be non-NULL", fn);
+  if ((rc = check_dtype(w_dtype, fn))) return rc;
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if ((rc = check_code(N, bits_per_pair, fn))) return rc;
+  if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
+  if (!std::isfinite(alpha)) return fail(QAMW_EINVAL, "%s: alpha must be finite", fn);
+  if (search_table != nullptr) return fail(QAMW_EUNSUPPORTED, "%s: search tables are not built yet", fn);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = launch_channel_scale(ScaleArgs{act_rms, alpha, K, col_scale_out, status}, st)) != cudaSuccess)
+    return cuda_fail(e, fn);
+  if ((e = launch_row_norms(RowNormArgs{W, w_dtype, M, K, ldw, col_scale_out, row_norm_out, status}, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, fn);
+  EncodeArgs ea;
+  ea.rot = RotateArgs{W, w_dtype, M, K, ldw, log2i(block), sign_seed, col_scale_out, row_norm_out};
+  ea.sigma = sigma;
+  ea.codebook = codebook;
+  ea.N = N;
+  ea.bits = bits_per_pair;
+  ea.wpr = qamw_words_per_row(K, bits_per_pair);
+  ea.packed = packed_out;
+  ea.status = status;
+  if ((e = launch_encode(ea, st)) != cudaSuccess) return cuda_fail(e, fn);
+  return QAMW_OK;
+}
+
+int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
+                int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
+                int32_t bits_per_pair, void *W_out, qamw_dtype out_dtype, int64_t ldo, int32_t *status,
+                qamw_stream_t stream) {
+  static const char *fn = "qamw_decode";
+  g_last_error[0] = 0;
+  int rc;
+  if (!packed || !row_norm || !sigma || !codebook || !W_out)
+    return fail(QAMW_ENULL, "%s: packed, row_norm, sigma, codebook, W_out must be non-NULL", fn);
+  if ((rc = check_dtype(out_dtype, fn))) return rc;
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if ((rc = check_code(N, bits_per_pair, fn))) return rc;
+  if (ldo < K) return fail(QAMW_EINVAL, "%s: ldo (%lld) < K (%lld)", fn, (long long)ldo, (long long)K);
+  DecodeArgs a;
+  a.packed = packed;
+  a.row_norm = row_norm;
+  a.sigma = sigma;
+  a.col_scale = col_scale;
+  a.M = M;
+  a.K = K;
+  a.log2b = log2i(block);
+  a.seed = sign_seed;
+  a.codebook = codebook;
+  a.N = N;
+  a.bits = bits_per_pair;
+  a.wpr = qamw_words_per_row(K, bits_per_pair);
+  a.out = W_out;
+  a.out_t = out_dtype;
+  a.ldo = ldo;
+  a.status = status;
+  cudaError_t e = launch_decode(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t block, uint64_t sign_seed,
+                     int32_t inverse, qamw_stream_t stream) {
+  static const char *fn = "qamw_rotate_rows";
+  g_last_error[0] = 0;
+  int rc;
+  if (!U || !Y) return fail(QAMW_ENULL, "%s: U and Y must be non-NULL", fn);
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  RotateTestArgs a{U, Y, M, K, log2i(block), sign_seed, inverse};
+  cudaError_t e = launch_rotate_test(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+}  // extern "C"

@@ -1,0 +1,443 @@
+// qamw_decode_tma.cu -- the bf16 decode with Tensor Memory Accelerator I/O.
+//
+// Same arithmetic as qamw_decode.cu ("QAM-W: Joint 2D Codebook Quantization
+// for LLM Weights ...", Methodology (6) Decoding), different data movement:
+//   * packed words reach shared memory through one 2D TMA tensor load per
+//     task (a box of ROWS rows x SEGS*128 columns worth of words), double
+//     buffered and tracked by an mbarrier per stage;
+//   * bf16 results are written into a 128-byte-swizzled staging tile and leave
+//     through 2D TMA tensor stores (one per 64 columns), which clip rows and
+//     columns past the matrix.
+// Neither transfer occupies the load/store unit, which profiling showed to be
+// the limiter of the plain-load / plain-store kernel (scattered 8-byte word
+// loads touched one sector per lane; the coalescing copy-out doubled the
+// shared-memory traffic of the staging).
+//
+// Task geometry: a warp decodes ROWS rows x SEGS segments of 128 columns with
+// lane = row + ROWS * segment. SEGS = b/128 for b > 128; otherwise 1, or 2
+// when one segment's words (8*bits bytes) are not a multiple of 16 bytes
+// (a TMA box row must be). Each lane owns one segment of one row, as in the
+// plain kernel.
+//
+// Every mbarrier wait is bounded; a wait that runs out sets
+// QAMW_STATUS_TIMEOUT and the kernel stops issuing work.
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "qamw_device.cuh"
+#include "qamw_internal.h"
+
+namespace qamw {
+namespace {
+
+constexpr int kSeg = 128;
+constexpr int kMaxWarps = 12;
+constexpr uint32_t kWaitLimit = 1u << 22;   // try_wait attempts before giving up
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; returns false if the phase did not complete in time.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, const void *src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+               "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+template <int BITS>
+__device__ __forceinline__ uint32_t extract_off8(const uint32_t *w, int q) {
+  constexpr uint32_t mask8 = ((1u << BITS) - 1u) << 3;
+  const int o = q * BITS, wi = o >> 5, sh = o & 31;
+  if (sh + BITS <= 32) {
+    if (sh >= 3) return (w[wi] >> (sh - 3)) & mask8;
+    return (w[wi] << (3 - sh)) & mask8;
+  }
+  return __funnelshift_r(w[wi], w[wi + 1], sh - 3) & mask8;
+}
+
+template <int TB>
+__device__ __forceinline__ void bfly_stage(float (&v)[kSeg]) {
+  constexpr int h = 1 << TB;
+#pragma unroll
+  for (int i = 0; i < kSeg; i += 2) {
+    if ((i & h) == 0) {
+      const float2 A = make_float2(v[i], v[i + 1]);
+      const float2 B = make_float2(v[i | h], v[(i | h) + 1]);
+      const float2 s = add2(A, B), d = sub2(A, B);
+      v[i] = s.x; v[i + 1] = s.y;
+      v[i | h] = d.x; v[(i | h) + 1] = d.y;
+    }
+  }
+}
+
+template <int LB>
+__device__ __forceinline__ void inlane_stages(float (&v)[kSeg]) {
+  if constexpr (LB > 1) bfly_stage<1>(v);
+  if constexpr (LB > 2) bfly_stage<2>(v);
+  if constexpr (LB > 3) bfly_stage<3>(v);
+  if constexpr (LB > 4) bfly_stage<4>(v);
+  if constexpr (LB > 5) bfly_stage<5>(v);
+  if constexpr (LB > 6) bfly_stage<6>(v);
+}
+
+template <int TB, int ROWS>
+__device__ __forceinline__ void xlane_stage(float (&v)[kSeg], int lane) {
+  constexpr int h = ROWS << (TB - 7);
+  const bool upper = (lane & h) != 0;
+#pragma unroll
+  for (int i = 0; i < kSeg; ++i) {
+    const float p = __shfl_xor_sync(0xffffffffu, v[i], h);
+    v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+  }
+}
+
+template <int LB, int ROWS>
+__device__ __forceinline__ void xlane_stages(float (&v)[kSeg], int lane) {
+  if constexpr (LB > 7) xlane_stage<7, ROWS>(v, lane);
+  if constexpr (LB > 8) xlane_stage<8, ROWS>(v, lane);
+  if constexpr (LB > 9) xlane_stage<9, ROWS>(v, lane);
+}
+
+template <int BITS, int LB>
+struct TmaGeom {
+  static constexpr int kSegs = (LB > 7) ? (1 << (LB - 7)) : ((BITS & 1) ? 2 : 1);
+  static constexpr int kRows = 32 / kSegs;
+  static constexpr int kLog2Rows = (kRows == 32) ? 5 : (kRows == 16) ? 4 : (kRows == 8) ? 3 : 2;
+  static constexpr int kBoxWords = kSegs * 2 * BITS;          // words per row of the input box
+  static constexpr int kInBytes = kRows * kBoxWords * 4;      // one input stage
+  static constexpr int kOutBoxes = kSegs * 2;                 // 64-column output boxes per task
+  static constexpr int kOutBoxBytes = kRows * 128;            // one swizzled output box
+  // per-warp layout (byte offsets); the staging tile first (1024-byte aligned)
+  static constexpr int kOffStage = 0;
+  static constexpr int kOffIn = kOffStage + kOutBoxes * kOutBoxBytes;
+  static constexpr int kOffCf = kOffIn + 2 * kInBytes;                 // kSegs x (128 + 4) floats
+  static constexpr int kOffSg = kOffCf + kSegs * (kSeg + 4) * 4;       // kSegs x (64 + 2) float2
+  static constexpr int kOffBar = kOffSg + kSegs * (kSeg / 2 + 2) * 8;  // 2 mbarriers
+  static constexpr int kWarpBytes = (kOffBar + 16 + 1023) & ~1023;
+};
+
+struct TmaArgs {
+  DecodeArgs a;
+  int copies, log2copies;
+  int64_t n_segcols, n_bands, n_tasks;
+};
+
+template <int BITS, int LB>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
+    decode_tma_kernel(TmaArgs ta, const __grid_constant__ CUtensorMap in_map,
+                      const __grid_constant__ CUtensorMap out_map) {
+  using G = TmaGeom<BITS, LB>;
+  constexpr int SEGS = G::kSegs, ROWS = G::kRows, NW = 2 * BITS;
+  const DecodeArgs &a = ta.a;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  // per-warp regions first (1024-byte aligned: the swizzled TMA boxes need it;
+  // the launch reserves 1 KB of slack), then the codebook table
+  unsigned char *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  unsigned char *wb = base + (size_t)warp * G::kWarpBytes;
+  unsigned char *stage = wb + G::kOffStage;
+  uint32_t *inbuf = reinterpret_cast<uint32_t *>(wb + G::kOffIn);
+  float *cf = reinterpret_cast<float *>(wb + G::kOffCf);
+  float2 *sg = reinterpret_cast<float2 *>(wb + G::kOffSg);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(wb + G::kOffBar);
+  float2 *cbp = reinterpret_cast<float2 *>(base + (size_t)nwarps * G::kWarpBytes);
+
+  for (int c = threadIdx.x; c < a.N; c += blockDim.x) {
+    const float c0 = a.codebook[2 * c], c1 = a.codebook[2 * c + 1];
+    const float2 e = make_float2(__fadd_rn(c0, c1), __fsub_rn(c0, c1));
+    for (int r = 0; r < ta.copies; ++r) cbp[c * ta.copies + r] = e;
+  }
+  if (lane == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  const float2 *cbl = cbp + (lane & (ta.copies - 1));
+  const int lgc = ta.log2copies;
+  const int rr = lane & (ROWS - 1);
+  const int sgi = lane >> G::kLog2Rows;
+  const int64_t gw = (int64_t)blockIdx.x * nwarps + warp;
+  const int64_t GW = (int64_t)gridDim.x * nwarps;
+  const int64_t t0 = gw * ta.n_tasks / GW, t1 = (gw + 1) * ta.n_tasks / GW;
+  const double inv_sqrt_b = 1.0 / sqrt((double)(1 << LB));
+  const int64_t P = a.K >> 1;
+  const bool check_idx = a.N < (1 << BITS);
+  uint32_t bad = 0;
+  bool timed_out = false;
+  int64_t cur = -1;
+
+  auto issue_load = [&](int64_t t, int st) {
+    const int64_t sc = t / ta.n_bands, bd = t - sc * ta.n_bands;
+    mbar_arrive_expect_tx(&bars[st], (uint32_t)G::kInBytes);
+    tma_load_2d(inbuf + st * (G::kInBytes / 4), &in_map, (int)(sc * G::kBoxWords), (int)(bd * ROWS), &bars[st]);
+  };
+  if (lane == 0 && t0 < t1) issue_load(t0, 0);
+
+  for (int64_t t = t0; t < t1; ++t) {
+    const int64_t segcol = t / ta.n_bands, band = t - segcol * ta.n_bands;
+    const int64_t colbase = segcol * (SEGS * kSeg);
+    const int st = (int)((t - t0) & 1);
+    const uint32_t parity = (uint32_t)(((t - t0) >> 1) & 1);
+    if (lane == 0 && t + 1 < t1) {
+      fence_proxy_async();   // stage st^1 was read by this warp in the previous task
+      issue_load(t + 1, st ^ 1);
+    }
+    if (segcol != cur) {
+      for (int j = lane; j < SEGS * kSeg; j += 32) {
+        const int64_t col = colbase + j;
+        float f = 0.0f;
+        if (col < a.K) {
+          const double s = (a.col_scale != nullptr) ? (double)a.col_scale[col] : 1.0;
+          double v = inv_sqrt_b / s;
+          if (mask_is_negative(a.seed, col)) v = -v;
+          f = (float)v;
+        }
+        cf[(j >> 7) * (kSeg + 4) + (j & 127)] = f;
+      }
+      for (int p = lane; p < SEGS * kSeg / 2; p += 32) {
+        const int64_t k = (colbase >> 1) + p;
+        const float sk = (k < P) ? a.sigma[k] : 0.0f;
+        sg[(p >> 6) * (kSeg / 2 + 2) + (p & 63)] = make_float2(sk, sk);
+      }
+      __syncwarp();
+      cur = segcol;
+    }
+    const int64_t row = band * ROWS + rr;
+    const bool row_ok = row < a.M;
+    float rn = 0.0f;
+    if (row_ok) {
+      rn = __ldg(a.row_norm + row);
+      if (!isfinite(rn)) bad |= QAMW_STATUS_NONFINITE_NORM;
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], parity))) {
+      timed_out = true;
+      break;
+    }
+    // words of this lane's segment
+    uint32_t w[NW + 1];
+    const uint32_t *wsrc = inbuf + st * (G::kInBytes / 4) + rr * G::kBoxWords + sgi * NW;
+#pragma unroll
+    for (int i = 0; i < NW / 2; ++i) {
+      const uint2 u = *reinterpret_cast<const uint2 *>(wsrc + 2 * i);
+      w[2 * i] = u.x;
+      w[2 * i + 1] = u.y;
+    }
+    w[NW] = 0u;
+    const int64_t col0 = colbase + (int64_t)sgi * kSeg;
+    const int vp = (int)std::min<int64_t>(kSeg, std::max<int64_t>(0, a.K - col0)) >> 1;
+    const float2 rn2 = make_float2(rn, rn);
+    const float2 *sgl = sg + sgi * (kSeg / 2 + 2);
+    float v[kSeg];
+    if (check_idx) {
+#pragma unroll
+      for (int q = 0; q < kSeg / 2; ++q) {
+        uint32_t off = extract_off8<BITS>(w, q);
+        if ((off >> 3) >= (uint32_t)a.N) {
+          if (row_ok && q < vp) bad |= QAMW_STATUS_BAD_INDEX;
+          off = 0;
+        }
+        const float2 y = mul2(mul2(sgl[q], rn2),
+                              *reinterpret_cast<const float2 *>(reinterpret_cast<const unsigned char *>(cbl) + (off << lgc)));
+        v[2 * q] = y.x;
+        v[2 * q + 1] = y.y;
+      }
+    } else {
+      const unsigned char *cbb = reinterpret_cast<const unsigned char *>(cbl);
+#pragma unroll
+      for (int q = 0; q < kSeg / 2; ++q) {
+        const uint32_t off = extract_off8<BITS>(w, q) << lgc;
+        const float2 y = mul2(mul2(sgl[q], rn2), *reinterpret_cast<const float2 *>(cbb + off));
+        v[2 * q] = y.x;
+        v[2 * q + 1] = y.y;
+      }
+    }
+    inlane_stages<LB>(v);
+    xlane_stages<LB, ROWS>(v, lane);
+
+    // the previous task's stores must have finished reading the staging tile
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+    const float *cfl = cf + sgi * (kSeg + 4);
+#pragma unroll
+    for (int c = 0; c < kSeg; c += 8) {
+      const float4 f0 = *reinterpret_cast<const float4 *>(cfl + c);
+      const float4 f1 = *reinterpret_cast<const float4 *>(cfl + c + 4);
+      const float2 o0 = mul2(make_float2(v[c], v[c + 1]), make_float2(f0.x, f0.y));
+      const float2 o1 = mul2(make_float2(v[c + 2], v[c + 3]), make_float2(f0.z, f0.w));
+      const float2 o2 = mul2(make_float2(v[c + 4], v[c + 5]), make_float2(f1.x, f1.y));
+      const float2 o3 = mul2(make_float2(v[c + 6], v[c + 7]), make_float2(f1.z, f1.w));
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(o0.x, o0.y);
+      __nv_bfloat162 b1 = __floats2bfloat162_rn(o1.x, o1.y);
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(o2.x, o2.y);
+      __nv_bfloat162 b3 = __floats2bfloat162_rn(o3.x, o3.y);
+      uint4 pk;
+      pk.x = *reinterpret_cast<uint32_t *>(&b0);
+      pk.y = *reinterpret_cast<uint32_t *>(&b1);
+      pk.z = *reinterpret_cast<uint32_t *>(&b2);
+      pk.w = *reinterpret_cast<uint32_t *>(&b3);
+      // column c of this lane's segment -> output box 2*sgi + c/64, 16-byte chunk (c%64)/8,
+      // stored at chunk ^ (row % 8) (the 128-byte swizzle of the TMA box)
+      const int box = 2 * sgi + (c >> 6);
+      const int chunk = ((c & 63) >> 3) ^ (rr & 7);
+      *reinterpret_cast<uint4 *>(stage + box * G::kOutBoxBytes + rr * 128 + chunk * 16) = pk;
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int bx = 0; bx < G::kOutBoxes; ++bx)
+        if (colbase + 64 * bx < a.K)
+          tma_store_2d(&out_map, (int)(colbase + 64 * bx), (int)(band * ROWS), stage + bx * G::kOutBoxBytes);
+      bulk_commit();
+    }
+    __syncwarp();
+  }
+  if (lane == 0) bulk_wait_all();
+  if (timed_out) bad |= QAMW_STATUS_TIMEOUT;
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  if (lane == 0) status_or(a.status, bad);
+}
+
+// --------------------------------------------------------------------------
+// host side
+// --------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+template <int BITS, int LB>
+cudaError_t launch_tma_t(const DecodeArgs &a, cudaStream_t s) {
+  using G = TmaGeom<BITS, LB>;
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  CUtensorMap in_map, out_map;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)a.wpr, (cuuint64_t)a.M};
+    cuuint64_t strides[1] = {(cuuint64_t)a.wpr * 4};
+    cuuint32_t box[2] = {(cuuint32_t)G::kBoxWords, (cuuint32_t)G::kRows};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&in_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(a.packed), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
+    cuuint64_t strides[1] = {(cuuint64_t)a.ldo * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)G::kRows};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&out_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
+  TmaArgs ta;
+  ta.a = a;
+  ta.copies = 16;
+  while (ta.copies > 1 && (size_t)a.N * 8 * ta.copies > 65536) ta.copies >>= 1;
+  int dev = 0, smem_max = 0;
+  cudaGetDevice(&dev);
+  cudaError_t e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  int warps = kMaxWarps;
+  auto need = [&](int w, int copies) { return 1024 + (size_t)w * G::kWarpBytes + (size_t)a.N * copies * 8; };
+  // prefer 12 warps; shrink the table replication, then the warp count, to fit
+  while (need(warps, ta.copies) > (size_t)smem_max && ta.copies > 4) ta.copies >>= 1;
+  while (warps > 4 && need(warps, ta.copies) > (size_t)smem_max) --warps;
+  while (need(warps, ta.copies) > (size_t)smem_max && ta.copies > 1) ta.copies >>= 1;
+  if (need(warps, ta.copies) > (size_t)smem_max) return cudaErrorNotSupported;
+  ta.log2copies = 0;
+  while ((1 << ta.log2copies) < ta.copies) ++ta.log2copies;
+  ta.n_segcols = (a.K + G::kSegs * kSeg - 1) / (G::kSegs * kSeg);
+  ta.n_bands = (a.M + G::kRows - 1) / G::kRows;
+  ta.n_tasks = ta.n_segcols * ta.n_bands;
+  const size_t smem = need(warps, ta.copies);
+  e = cudaFuncSetAttribute(decode_tma_kernel<BITS, LB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((ta.n_tasks + warps - 1) / warps, sm_count()));
+  decode_tma_kernel<BITS, LB><<<(int)blocks, warps * 32, smem, s>>>(ta, in_map, out_map);
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_tma_bits(const DecodeArgs &a, cudaStream_t s) {
+  switch (a.log2b) {
+    case 6: return launch_tma_t<BITS, 6>(a, s);
+    case 7: return launch_tma_t<BITS, 7>(a, s);
+    case 8: return launch_tma_t<BITS, 8>(a, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace
+
+bool decode_tma_applicable(const DecodeArgs &a) {
+  if (a.out_t != QAMW_BF16) return false;
+  if (a.bits != 7 && a.bits != 8 && a.bits != 10 && a.bits != 11) return false;
+  if (a.log2b < 6 || a.log2b > 8) return false;
+  if (reinterpret_cast<uintptr_t>(a.packed) % 16 || reinterpret_cast<uintptr_t>(a.out) % 16) return false;
+  if ((a.wpr * 4) % 16 || (a.ldo * 2) % 16) return false;
+  if (a.K % 64) return false;
+  if (a.M > (int64_t(1) << 31) || a.wpr > (int64_t(1) << 31)) return false;
+  return tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_decode_tma(const DecodeArgs &a, cudaStream_t s) {
+  switch (a.bits) {
+    case 7: return launch_tma_bits<7>(a, s);
+    case 8: return launch_tma_bits<8>(a, s);
+    case 10: return launch_tma_bits<10>(a, s);
+    case 11: return launch_tma_bits<11>(a, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace qamw

@@ -1,0 +1,105 @@
+// qamw_internal.h -- launcher interface between the C-ABI layer (qamw_api.cu)
+// and the kernel translation units. Arguments here are already validated.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "qamw.h"
+
+namespace qamw {
+
+// Rows per calibration row group (fixed, so the fp64 reduction order -- and
+// hence sigma -- does not depend on the device or the grid size).
+constexpr int kCalibRowGroup = 4;
+// Columns handled by one warp in the encode / calibrate kernels (32 lanes x 32).
+constexpr int kUnitCols = 1024;
+
+struct ScaleArgs {
+  const float *act_rms;  // [K] or nullptr
+  float alpha;
+  int64_t K;
+  float *s_out;          // [K]
+  int32_t *status;
+};
+
+struct RowNormArgs {
+  const void *W;
+  qamw_dtype wt;
+  int64_t M, K, ldw;
+  const float *s;        // [K]
+  float *r_out;          // [M]
+  int32_t *status;
+};
+
+struct RotateArgs {       // shared by encode and calibrate
+  const void *W;
+  qamw_dtype wt;
+  int64_t M, K, ldw;
+  int32_t log2b;
+  uint64_t seed;
+  const float *s;        // [K] channel scales
+  const float *r;        // [M] stored row norms
+};
+
+struct CalibArgs {
+  RotateArgs rot;
+  double *partials;      // [G][K/2]
+  int64_t groups;        // G = ceil(M / kCalibRowGroup)
+  float *sigma_out;      // [K/2]
+};
+
+struct EncodeArgs {
+  RotateArgs rot;
+  const float *sigma;    // [K/2]
+  const float *codebook; // [N][2]
+  int32_t N;
+  int32_t bits;
+  int64_t wpr;           // words per row
+  uint32_t *packed;      // [M][wpr]
+  int32_t *status;
+};
+
+struct DecodeArgs {
+  const uint32_t *packed;
+  const float *row_norm;
+  const float *sigma;
+  const float *col_scale;  // nullable
+  int64_t M, K;
+  int32_t log2b;
+  uint64_t seed;
+  const float *codebook;
+  int32_t N;
+  int32_t bits;
+  int64_t wpr;
+  void *out;
+  qamw_dtype out_t;
+  int64_t ldo;
+  int32_t *status;
+};
+
+struct RotateTestArgs {
+  const double *U;
+  double *Y;
+  int64_t M, K;
+  int32_t log2b;
+  uint64_t seed;
+  int32_t inverse;
+};
+
+// Each launcher returns cudaSuccess or the launch error.
+cudaError_t launch_channel_scale(const ScaleArgs &a, cudaStream_t s);
+cudaError_t launch_row_norms(const RowNormArgs &a, cudaStream_t s);
+cudaError_t launch_calibrate(const CalibArgs &a, cudaStream_t s);
+cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// bf16 decode with TMA tensor loads/stores (qamw_decode_tma.cu).
+bool decode_tma_applicable(const DecodeArgs &a);
+cudaError_t launch_decode_tma(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_rotate_test(const RotateTestArgs &a, cudaStream_t s);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+}  // namespace qamw
