@@ -134,6 +134,11 @@ __device__ __forceinline__ void xlane_stages(float (&v)[kSeg], int lane) {
   if constexpr (LB > 9) xlane_stage<9, ROWS>(v, lane);
 }
 
+#ifndef QAMW_DEC_STAGES
+#define QAMW_DEC_STAGES 1
+#endif
+constexpr int kStages = QAMW_DEC_STAGES;   // input pipeline depth; 1 measured fastest (more stages cost warps)
+
 template <int BITS, int LB>
 struct TmaGeom {
   static constexpr int kSegs = (LB > 7) ? (1 << (LB - 7)) : ((BITS & 1) ? 2 : 1);
@@ -146,10 +151,11 @@ struct TmaGeom {
   // per-warp layout (byte offsets); the staging tile first (1024-byte aligned)
   static constexpr int kOffStage = 0;
   static constexpr int kOffIn = kOffStage + kOutBoxes * kOutBoxBytes;
-  static constexpr int kOffCf = kOffIn + 2 * kInBytes;                 // kSegs x (128 + 4) floats
+  static constexpr int kStageBytes = kInBytes + ((kRows * 4 + 127) & ~127);  // words + row norms
+  static constexpr int kOffCf = kOffIn + kStages * kStageBytes;        // kSegs x (128 + 4) floats
   static constexpr int kOffSg = kOffCf + kSegs * (kSeg + 4) * 4;       // kSegs x (64 + 2) float2
-  static constexpr int kOffBar = kOffSg + kSegs * (kSeg / 2 + 2) * 8;  // 2 mbarriers
-  static constexpr int kWarpBytes = (kOffBar + 16 + 1023) & ~1023;
+  static constexpr int kOffBar = kOffSg + kSegs * (kSeg / 2 + 2) * 8;  // kStages mbarriers
+  static constexpr int kWarpBytes = (kOffBar + 8 * kStages + 1023) & ~1023;
 };
 
 struct TmaArgs {
@@ -161,7 +167,7 @@ struct TmaArgs {
 template <int BITS, int LB>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     decode_tma_kernel(TmaArgs ta, const __grid_constant__ CUtensorMap in_map,
-                      const __grid_constant__ CUtensorMap out_map) {
+                      const __grid_constant__ CUtensorMap rn_map, const __grid_constant__ CUtensorMap out_map) {
   using G = TmaGeom<BITS, LB>;
   constexpr int SEGS = G::kSegs, ROWS = G::kRows, NW = 2 * BITS;
   const DecodeArgs &a = ta.a;
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   unsigned char *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char *wb = base + (size_t)warp * G::kWarpBytes;
   unsigned char *stage = wb + G::kOffStage;
-  uint32_t *inbuf = reinterpret_cast<uint32_t *>(wb + G::kOffIn);
+  unsigned char *inbase = wb + G::kOffIn;   // stage st: words, then row norms
   float *cf = reinterpret_cast<float *>(wb + G::kOffCf);
   float2 *sg = reinterpret_cast<float2 *>(wb + G::kOffSg);
   uint64_t *bars = reinterpret_cast<uint64_t *>(wb + G::kOffBar);
@@ -185,8 +191,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     for (int r = 0; r < ta.copies; ++r) cbp[c * ta.copies + r] = e;
   }
   if (lane == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -195,32 +200,54 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
   const int lgc = ta.log2copies;
   const int rr = lane & (ROWS - 1);
   const int sgi = lane >> G::kLog2Rows;
-  const int64_t gw = (int64_t)blockIdx.x * nwarps + warp;
-  const int64_t GW = (int64_t)gridDim.x * nwarps;
-  const int64_t t0 = gw * ta.n_tasks / GW, t1 = (gw + 1) * ta.n_tasks / GW;
+  // Work split: warp g keeps column strip g % n_strips for its whole life (its
+  // column tables are built once) and takes the bands slot, slot + per_strip,
+  // slot + 2 per_strip, ... with slot = g / n_strips. All warps therefore move
+  // down the matrix together and the reads and writes of any moment fall in
+  // one band of consecutive rows, which keeps DRAM pages open; giving each
+  // warp a contiguous run of tasks instead scattered the writes over the whole
+  // matrix and halved the store throughput.
+  const int gw = blockIdx.x * nwarps + warp;
+  const int GW = gridDim.x * nwarps;
+  const int nsc = (int)ta.n_segcols, nb = (int)ta.n_bands;
+  const int per_strip = GW / nsc;           // >= 1 (checked on the host)
+  const int my_strip = gw % nsc, slot = gw / nsc;
+  const bool active = slot < per_strip;
+  // tasks of this warp: k = 0, 1, ... with band = slot + k * per_strip
+  const int t0 = 0, t1 = active ? (nb - slot + per_strip - 1) / per_strip : 0;
   const double inv_sqrt_b = 1.0 / sqrt((double)(1 << LB));
   const int64_t P = a.K >> 1;
   const bool check_idx = a.N < (1 << BITS);
   uint32_t bad = 0;
   bool timed_out = false;
-  int64_t cur = -1;
+  int cur = -1;
 
-  auto issue_load = [&](int64_t t, int st) {
-    const int64_t sc = t / ta.n_bands, bd = t - sc * ta.n_bands;
-    mbar_arrive_expect_tx(&bars[st], (uint32_t)G::kInBytes);
-    tma_load_2d(inbuf + st * (G::kInBytes / 4), &in_map, (int)(sc * G::kBoxWords), (int)(bd * ROWS), &bars[st]);
+  // Input pipeline: kStages buffers of (packed words, row norms). The prologue
+  // fills all of them; as soon as every lane has copied task t's words to
+  // registers, its buffer is reloaded with task t + kStages, so each load has
+  // about kStages tasks of compute time to arrive.
+  auto issue_load = [&](int t) {
+    const int st = (t - t0) % kStages;
+    const int sc = my_strip, bd = slot + t * per_strip;
+    unsigned char *buf = inbase + st * G::kStageBytes;
+    mbar_arrive_expect_tx(&bars[st], (uint32_t)(G::kInBytes + ROWS * 4));
+    tma_load_2d(buf, &in_map, sc * G::kBoxWords, bd * ROWS, &bars[st]);
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];" ::"r"(
+            smem_u32(buf + G::kInBytes)),
+        "l"(&rn_map), "r"(bd * ROWS), "r"(smem_u32(&bars[st]))
+        : "memory");
   };
-  if (lane == 0 && t0 < t1) issue_load(t0, 0);
+  if (lane == 0)
+    for (int t = t0; t < t1 && t < t0 + kStages; ++t) issue_load(t);
 
-  for (int64_t t = t0; t < t1; ++t) {
-    const int64_t segcol = t / ta.n_bands, band = t - segcol * ta.n_bands;
-    const int64_t colbase = segcol * (SEGS * kSeg);
-    const int st = (int)((t - t0) & 1);
-    const uint32_t parity = (uint32_t)(((t - t0) >> 1) & 1);
-    if (lane == 0 && t + 1 < t1) {
-      fence_proxy_async();   // stage st^1 was read by this warp in the previous task
-      issue_load(t + 1, st ^ 1);
-    }
+  for (int t = t0; t < t1; ++t) {
+    const int segcol = my_strip, band = slot + t * per_strip;
+    const int64_t colbase = (int64_t)segcol * (SEGS * kSeg);
+    const int st = (t - t0) % kStages;
+    const uint32_t parity = (uint32_t)(((t - t0) / kStages) & 1);
+    const uint32_t *inbuf = reinterpret_cast<const uint32_t *>(inbase + st * G::kStageBytes);
+    const float *rnbuf = reinterpret_cast<const float *>(inbase + st * G::kStageBytes + G::kInBytes);
     if (segcol != cur) {
       for (int j = lane; j < SEGS * kSeg; j += 32) {
         const int64_t col = colbase + j;
@@ -241,20 +268,20 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       __syncwarp();
       cur = segcol;
     }
-    const int64_t row = band * ROWS + rr;
-    const bool row_ok = row < a.M;
-    float rn = 0.0f;
-    if (row_ok) {
-      rn = __ldg(a.row_norm + row);
-      if (!isfinite(rn)) bad |= QAMW_STATUS_NONFINITE_NORM;
-    }
     if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], parity))) {
       timed_out = true;
       break;
     }
+    const int64_t row = (int64_t)band * ROWS + rr;
+    const bool row_ok = row < a.M;
+    float rn = 0.0f;
+    if (row_ok) {
+      rn = rnbuf[rr];
+      if (!isfinite(rn)) bad |= QAMW_STATUS_NONFINITE_NORM;
+    }
     // words of this lane's segment
     uint32_t w[NW + 1];
-    const uint32_t *wsrc = inbuf + st * (G::kInBytes / 4) + rr * G::kBoxWords + sgi * NW;
+    const uint32_t *wsrc = inbuf + rr * G::kBoxWords + sgi * NW;
 #pragma unroll
     for (int i = 0; i < NW / 2; ++i) {
       const uint2 u = *reinterpret_cast<const uint2 *>(wsrc + 2 * i);
@@ -262,6 +289,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       w[2 * i + 1] = u.y;
     }
     w[NW] = 0u;
+    __syncwarp();
+    if (lane == 0 && t + kStages < t1) {
+      fence_proxy_async();
+      issue_load(t + kStages);
+    }
     const int64_t col0 = colbase + (int64_t)sgi * kSeg;
     const int vp = (int)std::min<int64_t>(kSeg, std::max<int64_t>(0, a.K - col0)) >> 1;
     const float2 rn2 = make_float2(rn, rn);
@@ -326,7 +358,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 #pragma unroll
       for (int bx = 0; bx < G::kOutBoxes; ++bx)
         if (colbase + 64 * bx < a.K)
-          tma_store_2d(&out_map, (int)(colbase + 64 * bx), (int)(band * ROWS), stage + bx * G::kOutBoxBytes);
+          tma_store_2d(&out_map, (int)(colbase + 64 * bx), band * ROWS, stage + bx * G::kOutBoxBytes);
       bulk_commit();
     }
     __syncwarp();
@@ -358,7 +390,17 @@ cudaError_t launch_tma_t(const DecodeArgs &a, cudaStream_t s) {
   using G = TmaGeom<BITS, LB>;
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
-  CUtensorMap in_map, out_map;
+  CUtensorMap in_map, rn_map, out_map;
+  {
+    cuuint64_t dims[1] = {(cuuint64_t)a.M};
+    cuuint64_t strides[1] = {4};
+    cuuint32_t box[1] = {(cuuint32_t)G::kRows};
+    cuuint32_t es[1] = {1};
+    if (enc(&rn_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float *>(a.row_norm), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorNotSupported;
+  }
   {
     cuuint64_t dims[2] = {(cuuint64_t)a.wpr, (cuuint64_t)a.M};
     cuuint64_t strides[1] = {(cuuint64_t)a.wpr * 4};
@@ -402,8 +444,10 @@ cudaError_t launch_tma_t(const DecodeArgs &a, cudaStream_t s) {
   const size_t smem = need(warps, ta.copies);
   e = cudaFuncSetAttribute(decode_tma_kernel<BITS, LB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // one CTA per SM; every column strip needs at least one warp
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((ta.n_tasks + warps - 1) / warps, sm_count()));
-  decode_tma_kernel<BITS, LB><<<(int)blocks, warps * 32, smem, s>>>(ta, in_map, out_map);
+  if (blocks * warps < ta.n_segcols) return cudaErrorNotSupported;
+  decode_tma_kernel<BITS, LB><<<(int)blocks, warps * 32, smem, s>>>(ta, in_map, rn_map, out_map);
   return cudaGetLastError();
 }
 
@@ -426,7 +470,11 @@ bool decode_tma_applicable(const DecodeArgs &a) {
   if (reinterpret_cast<uintptr_t>(a.packed) % 16 || reinterpret_cast<uintptr_t>(a.out) % 16) return false;
   if ((a.wpr * 4) % 16 || (a.ldo * 2) % 16) return false;
   if (a.K % 64) return false;
-  if (a.M > (int64_t(1) << 31) || a.wpr > (int64_t(1) << 31)) return false;
+  if (a.M > (int64_t(1) << 30) || a.wpr > (int64_t(1) << 30)) return false;
+  if (reinterpret_cast<uintptr_t>(a.row_norm) % 16) return false;
+  // task indices are 32-bit
+  const int64_t segs = (a.log2b > 7) ? (int64_t(1) << (a.log2b - 7)) : ((a.bits & 1) ? 2 : 1);
+  if (((a.K + segs * 128 - 1) / (segs * 128)) * ((a.M + 31) / (32 / segs)) > (int64_t(1) << 30)) return false;
   return tensor_map_encoder() != nullptr;
 }
 
