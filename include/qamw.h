@@ -118,6 +118,38 @@ int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K
                          int32_t *status, qamw_stream_t stream);
 
 /*
+ * qamw_calibrate_sigma_noalloc -- qamw_calibrate_sigma for callers that cannot
+ * allocate device memory.
+ * (An interface of this library; the QAM-W page has no counterpart.)
+ * Some callers cannot provide the calibration workspace: an inference engine
+ * that freezes its device memory pool after start-up, a plug-in whose host
+ * framework owns all device memory and offers no allocator, or a
+ * latency-critical path on which cudaMalloc (which may synchronize the
+ * device) is not acceptable. This entry point computes exactly what
+ * qamw_calibrate_sigma computes, with the same arguments minus the
+ * workspace, using a fixed scratch area of QAMW_NOALLOC_SCRATCH_BYTES bytes
+ * built into the library; neither it nor the library allocates anything.
+ *   - Limit: qamw_calibrate_workspace_bytes(M, K) must not exceed
+ *     QAMW_NOALLOC_SCRATCH_BYTES (about M*K <= 33.5 million weights);
+ *     larger shapes return QAMW_EUNSUPPORTED with a message that says so.
+ *   - The area is reserved on every GPU that loads the library, until the
+ *     process exits.
+ *   - Set-up: the first call made with a given device current looks up the
+ *     area's device address (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture on that device.
+ *   - All calls share the one area and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each call writes every byte it
+ *     reads). Calls whose kernels overlap on the GPU (different streams, or
+ *     different host threads) race on the area: serialize them.
+ * Errors: as qamw_calibrate_sigma (except EWORKSPACE), plus QAMW_EUNSUPPORTED
+ * for shapes beyond the limit and QAMW_ECUDA if the address lookup fails.
+ */
+#define QAMW_NOALLOC_SCRATCH_BYTES (32u << 20)
+int qamw_calibrate_sigma_noalloc(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                                 const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                                 float *sigma_out, int32_t *status, qamw_stream_t stream);
+
+/*
  * qamw_encode -- Methodology steps (5), (1), (2), (3), (4) and bit packing.
  * For every row: s_j (step 5), r_i = RN32(||w' ||) written to row_norm_out
  * (step 1), the sign-masked block Hadamard rotation (step 2, in fp64, so that

@@ -50,6 +50,8 @@ _SIGNATURES = {
     "qamw_decode": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
                                    _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
+    "qamw_calibrate_sigma_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
+                                                    _c_i32, _c_u64, _c_p, _c_p, _c_p]),
 }
 
 _lib = None
@@ -105,6 +107,7 @@ qamw_calibrate_sigma = _raw("qamw_calibrate_sigma")
 qamw_encode = _raw("qamw_encode")
 qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
+qamw_calibrate_sigma_noalloc = _raw("qamw_calibrate_sigma_noalloc")
 
 
 # ---------------------------------------------------------------------------

@@ -70,6 +70,8 @@ std::mutex g_sm_mu;
 int g_sm_count[64] = {0};
 }  // namespace
 
+void set_last_error(const char *msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 int sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;

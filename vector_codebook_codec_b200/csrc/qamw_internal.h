@@ -102,4 +102,7 @@ cudaError_t launch_rotate_test(const RotateTestArgs &a, cudaStream_t s);
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Sets the message qamw_last_error() returns on this host thread.
+void set_last_error(const char *msg);
+
 }  // namespace qamw
