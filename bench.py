@@ -54,6 +54,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
+    p.add_argument("--search", choices=("pruned", "brute"), default="pruned",
+                   help="nearest-centroid search: exact pruned table (default) or brute force")
     return p.parse_args(argv)
 
 
@@ -356,6 +358,7 @@ def run_ours(args):
     Wd = Wt.to(dev)
     actd = torch.from_numpy(act).to(dev)
     Cd = torch.from_numpy(C).to(dev)
+    table = q.build_search_table(Cd) if args.search == "pruned" else None   # once per codebook
     lib = q.load_library()
     wpr = q.words_per_row(K, spec.bits)
     ws = torch.empty(int(lib.qamw_calibrate_workspace_bytes(M, K)), dtype=torch.uint8, device=dev)
@@ -376,7 +379,7 @@ def run_ours(args):
                                 out=sigma)
         if evs: evs[1].record(stream)
         enc = q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sig, Cd, spec.bits, status=status,
-                       out=(packed, rnorm, cscale))
+                       out=(packed, rnorm, cscale), search_table=table)
         if evs: evs[2].record(stream)
         q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=out)
         if evs: evs[3].record(stream)

@@ -176,6 +176,22 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
                 float *col_scale_out, int32_t *status, qamw_stream_t stream);
 
 /*
+ * qamw_search_table_bytes / qamw_build_search_table -- an exact pruned search
+ * for Methodology (4): a grid over the plane of normalised pairs, each cell
+ * listing (in ascending index order) every centroid that can be the fp32
+ * nearest one for a pair in that cell. qamw_encode given the table returns
+ * the same indices as without it (the brute-force search), faster. The table
+ * depends only on the codebook; build it once per codebook.
+ *   codebook : device float32 [N][2]      table: device, 16-byte aligned,
+ *   >= qamw_search_table_bytes(N) bytes (0 if N is out of range).
+ * A codebook whose lists overflow the table's capacity yields a table marked
+ * invalid, with which qamw_encode uses the brute-force search.
+ */
+size_t qamw_search_table_bytes(int32_t N);
+int qamw_build_search_table(const float *codebook, int32_t N, void *table, size_t table_bytes,
+                            qamw_stream_t stream);
+
+/*
  * qamw_decode -- Methodology (6) Decoding.
  * w_hat_ij = r_i * d_j * (H_b (sigma (.) C[idx]))_j / (sqrt(b) * s_j): unpack,
  * look up centroids, rescale by sigma_k, inverse rotation, multiply by the

@@ -98,7 +98,7 @@ def _cal(lib, **kw):
     (dict(bits=17), QAMW_EINVAL), (dict(N=257), QAMW_EINVAL), (dict(N=0), QAMW_EINVAL),
     (dict(N=16384, bits=16), QAMW_EUNSUPPORTED), (dict(alpha=float("nan")), QAMW_EINVAL),
     (dict(alpha=float("inf")), QAMW_EINVAL), (dict(wt=7), QAMW_EINVAL),
-    (dict(table=FAKE), QAMW_EUNSUPPORTED),
+    (dict(table=ctypes.c_void_p(0x10008)), QAMW_EINVAL),
 ])
 def test_encode_rejects_on_host(lib, kw, code):
     assert _enc(lib, **kw) == code

@@ -50,6 +50,8 @@ _SIGNATURES = {
     "qamw_decode": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
                                    _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
+    "qamw_search_table_bytes": (_c_sz, [_c_i32]),
+    "qamw_build_search_table": (ctypes.c_int, [_c_p, _c_i32, _c_p, _c_sz, _c_p]),
     "qamw_calibrate_sigma_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
                                                     _c_i32, _c_u64, _c_p, _c_p, _c_p]),
 }
@@ -108,6 +110,8 @@ qamw_encode = _raw("qamw_encode")
 qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
 qamw_calibrate_sigma_noalloc = _raw("qamw_calibrate_sigma_noalloc")
+qamw_search_table_bytes = _raw("qamw_search_table_bytes")
+qamw_build_search_table = _raw("qamw_build_search_table")
 
 
 # ---------------------------------------------------------------------------
@@ -214,9 +218,27 @@ class Encoded:
     bits: int
 
 
+def build_search_table(codebook, stream=None):
+    """Search table for the exact pruned search (uint8 CUDA tensor); build once per codebook."""
+    torch = _torch()
+    _need_cuda("codebook", codebook, torch.float32, 2)
+    N = codebook.shape[0]
+    lib = load_library()
+    nbytes = int(lib.qamw_search_table_bytes(N))
+    if nbytes == 0:
+        raise ValueError(f"no search table for N={N}")
+    table = torch.empty(nbytes, dtype=torch.uint8, device=codebook.device)
+    _check("qamw_build_search_table", lib.qamw_build_search_table(
+        _ptr(codebook.contiguous()), N, _ptr(table), nbytes, _stream_ptr(stream)))
+    return table
+
+
 def encode(W, act_rms, alpha: float, block: int, seed: int, sigma, codebook, bits: int,
-           status=None, stream=None, out=None) -> Encoded:
-    """Encode W with the given sigma and codebook (float32 CUDA tensor [N, 2])."""
+           status=None, stream=None, out=None, search_table=None) -> Encoded:
+    """Encode W with the given sigma and codebook (float32 CUDA tensor [N, 2]).
+
+    ``search_table`` (from :func:`build_search_table`) selects the exact pruned
+    search; without it every pair is compared with all N centroids."""
     torch = _torch()
     _need_cuda("W", W, ndim=2)
     _need_cuda("act_rms", act_rms, torch.float32, 1)
@@ -235,7 +257,7 @@ def encode(W, act_rms, alpha: float, block: int, seed: int, sigma, codebook, bit
         packed, r, s = out
     _check("qamw_encode", load_library().qamw_encode(
         _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
-        _ptr(sigma), _ptr(codebook.contiguous()), N, bits, None, _ptr(packed), _ptr(r), _ptr(s),
+        _ptr(sigma), _ptr(codebook.contiguous()), N, bits, _ptr(search_table), _ptr(packed), _ptr(r), _ptr(s),
         _ptr(status), _stream_ptr(stream)))
     return Encoded(packed, r, s, sigma, M, K, block, seed, N, bits)
 

@@ -178,7 +178,8 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
   if ((rc = check_code(N, bits_per_pair, fn))) return rc;
   if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
   if (!std::isfinite(alpha)) return fail(QAMW_EINVAL, "%s: alpha must be finite", fn);
-  if (search_table != nullptr) return fail(QAMW_EUNSUPPORTED, "%s: search tables are not built yet", fn);
+  if (search_table != nullptr && reinterpret_cast<uintptr_t>(search_table) % 16)
+    return fail(QAMW_EINVAL, "%s: search_table must be 16-byte aligned", fn);
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if ((e = launch_channel_scale(ScaleArgs{act_rms, alpha, K, col_scale_out, status}, st)) != cudaSuccess)
@@ -194,6 +195,7 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
   ea.bits = bits_per_pair;
   ea.wpr = qamw_words_per_row(K, bits_per_pair);
   ea.packed = packed_out;
+  ea.table = search_table;
   ea.status = status;
   if ((e = launch_encode(ea, st)) != cudaSuccess) return cuda_fail(e, fn);
   return QAMW_OK;
@@ -230,6 +232,25 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
   a.ldo = ldo;
   a.status = status;
   cudaError_t e = launch_decode(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+size_t qamw_search_table_bytes(int32_t N) {
+  if (N < 1 || N > QAMW_MAX_CENTROIDS) return 0;
+  return search_table_bytes(N);
+}
+
+int qamw_build_search_table(const float *codebook, int32_t N, void *table, size_t table_bytes,
+                            qamw_stream_t stream) {
+  static const char *fn = "qamw_build_search_table";
+  g_last_error[0] = 0;
+  if (!codebook || !table) return fail(QAMW_ENULL, "%s: codebook and table must be non-NULL", fn);
+  if (N < 1) return fail(QAMW_EINVAL, "%s: N must be >= 1 (got %d)", fn, N);
+  if (N > QAMW_MAX_CENTROIDS) return fail(QAMW_EUNSUPPORTED, "%s: N=%d exceeds %d", fn, N, QAMW_MAX_CENTROIDS);
+  const size_t need = search_table_bytes(N);
+  if (table_bytes < need) return fail(QAMW_EWORKSPACE, "%s: table of %zu bytes needed (got %zu)", fn, need, table_bytes);
+  if (reinterpret_cast<uintptr_t>(table) % 16) return fail(QAMW_EINVAL, "%s: table must be 16-byte aligned", fn);
+  cudaError_t e = launch_build_search_table(codebook, N, table, (cudaStream_t)stream);
   return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
 }
 

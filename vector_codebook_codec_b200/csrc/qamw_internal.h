@@ -16,6 +16,20 @@ constexpr int kCalibRowGroup = 4;
 // Columns handled by one warp in the encode / calibrate kernels (32 lanes x 32).
 constexpr int kUnitCols = 1024;
 
+// Header of a search table (see qamw_search.cu).
+constexpr uint32_t kSearchMagic = 0x54574D51u;   // "QMWT"
+struct SearchHeader {
+  uint32_t magic;
+  int32_t N, G, total;
+  float L, inv_cw;   // grid covers [-L, L]^2; cell index = floor((x + L) * inv_cw)
+  int32_t valid, capacity;
+};
+static_assert(sizeof(SearchHeader) == 32, "search header is 32 bytes");
+int search_grid(int N);
+int64_t search_capacity(int N);
+size_t search_table_bytes(int N);
+cudaError_t launch_build_search_table(const float *codebook, int N, void *table, cudaStream_t s);
+
 struct ScaleArgs {
   const float *act_rms;  // [K] or nullptr
   float alpha;
@@ -58,6 +72,7 @@ struct EncodeArgs {
   int32_t bits;
   int64_t wpr;           // words per row
   uint32_t *packed;      // [M][wpr]
+  const void *table;     // search table or nullptr (brute force)
   int32_t *status;
 };
 

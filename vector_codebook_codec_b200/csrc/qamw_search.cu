@@ -1,0 +1,202 @@
+// qamw_search.cu -- candidate table for the exact pruned nearest-centroid search.
+//
+// Methodology (4) Joint 2D Quantization of the QAM-W page maps each normalised
+// pair x to the nearest centroid of one 2D codebook. The brute-force search
+// computes N distances per pair. This table lets the encode compute only the
+// distances that can matter: x-space is cut into a G x G grid of cells over
+// [-L, L]^2 (L a little beyond the outermost centroid); for every cell Q
+// (enlarged by a small margin) the table lists every centroid c with
+//     dmin(c, Q)^2 <= (1 + 1e-5) * D(Q)^2,   D(Q) = min_c' dmax(c', Q),
+// dmin / dmax being the least / greatest distance from c to a point of Q.
+// For a pair x in Q its exact nearest distance d* is at most D(Q), and every
+// centroid whose fp32 direct-difference distance ties or beats the fp32
+// distance of the exact nearest one is within a factor (1 + 4e-7) of d*, so
+// it is listed. Scanning a cell's list in ascending index order with a strict
+// "<" therefore returns exactly the index of the brute-force search (the
+// lowest index among the fp32 minimisers). Pairs outside the grid, or a table
+// that does not fit, use the brute-force search.
+//
+// Table layout (device memory owned by the caller, 16-byte aligned):
+//   SearchHeader | uint32 offsets[G*G + 1] | uint16 cand[capacity]
+// cand[offsets[k] .. offsets[k+1]) are the centroid indices of cell
+// k = iy * G + ix in ascending order. The build is four kernels with a fixed
+// order of every reduction, so the table is a pure function of the codebook.
+#include <cfloat>
+#include <cmath>
+
+#include "qamw_device.cuh"
+#include "qamw_internal.h"
+
+namespace qamw {
+
+int search_grid(int N) { return N >= 1024 ? 128 : (N >= 128 ? 64 : 32); }
+
+int64_t search_capacity(int N) {
+  const int G = search_grid(N);
+  return (int64_t)G * G * (N < 64 ? N : 64);   // a cell lists at most N (and in practice far fewer than 64)
+}
+
+size_t search_table_bytes(int N) {
+  const int G = search_grid(N);
+  const size_t off = sizeof(SearchHeader) + (size_t)(G * G + 1) * 4;
+  return (off + (size_t)search_capacity(N) * 2 + 15) & ~size_t(15);
+}
+
+namespace {
+
+constexpr double kCellMargin = 1e-3;   // cell enlargement, in cells (covers fp32 rounding of the cell index)
+constexpr double kTieSlack = 1e-5;     // relative slack on D(Q)^2
+
+__global__ void table_header_kernel(const float *codebook, int N, int G, int64_t capacity, SearchHeader *h) {
+  __shared__ float red[32];
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < 2 * N; i += blockDim.x) m = fmaxf(m, fabsf(codebook[i]));
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+    const float L = r * 1.02f + 0.6f;
+    h->magic = kSearchMagic;
+    h->N = N;
+    h->G = G;
+    h->total = 0;
+    h->L = L;
+    h->inv_cw = (float)G / (2.0f * L);
+    h->valid = 0;
+    h->capacity = (int32_t)capacity;
+  }
+}
+
+// Enlarged bounds of cell (ix, iy) in fp64.
+__device__ __forceinline__ void cell_bounds(const SearchHeader &h, int cell, double &x0, double &x1, double &y0,
+                                            double &y1) {
+  const int ix = cell % h.G, iy = cell / h.G;
+  const double L = (double)h.L, cw = 2.0 * L / (double)h.G, m = kCellMargin * cw;
+  x0 = -L + ix * cw - m;
+  x1 = -L + (ix + 1) * cw + m;
+  y0 = -L + iy * cw - m;
+  y1 = -L + (iy + 1) * cw + m;
+}
+
+__device__ __forceinline__ double dmax2(double cx, double cy, double x0, double x1, double y0, double y1) {
+  const double ax = fmax(fabs(cx - x0), fabs(cx - x1)), ay = fmax(fabs(cy - y0), fabs(cy - y1));
+  return ax * ax + ay * ay;
+}
+__device__ __forceinline__ double dmin2(double cx, double cy, double x0, double x1, double y0, double y1) {
+  const double ax = fmax(0.0, fmax(x0 - cx, cx - x1)), ay = fmax(0.0, fmax(y0 - cy, cy - y1));
+  return ax * ax + ay * ay;
+}
+
+// D(Q)^2 * (1 + slack) for the warp's cell; every lane gets it.
+__device__ double cell_bound(const float *codebook, int N, double x0, double x1, double y0, double y1, int lane) {
+  double d = DBL_MAX;
+  for (int i = lane; i < N; i += 32) d = fmin(d, dmax2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1));
+  for (int o = 16; o > 0; o >>= 1) d = fmin(d, __shfl_xor_sync(0xffffffffu, d, o));
+  return d * (1.0 + kTieSlack);
+}
+
+__global__ void table_count_kernel(const float *codebook, SearchHeader *h, uint32_t *offsets) {
+  const int lane = threadIdx.x & 31;
+  const int cell = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+  const SearchHeader hh = *h;
+  if (cell >= hh.G * hh.G) return;
+  double x0, x1, y0, y1;
+  cell_bounds(hh, cell, x0, x1, y0, y1);
+  const double bound = cell_bound(codebook, hh.N, x0, x1, y0, y1, lane);
+  int cnt = 0;
+  for (int i = lane; i < hh.N; i += 32) cnt += dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) offsets[cell + 1] = (uint32_t)cnt;
+}
+
+// Prefix sum of the G*G counts held in offsets[1..n] (one CTA of 1024
+// threads, fixed order). Each thread owns up to kScanPer consecutive cells:
+// it keeps their counts in registers and writes only their offsets, so no
+// slot is read by one thread and written by another.
+constexpr int kScanPer = 16;   // 16384 cells (G = 128) / 1024 threads
+__global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint32_t *offsets) {
+  __shared__ uint32_t wsum[32];
+  const int n = h->G * h->G;
+  const int b = threadIdx.x * kScanPer;
+  uint32_t cnt[kScanPer];
+  uint32_t s = 0;
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k) {
+    cnt[k] = (b + k < n) ? offsets[b + k + 1] : 0u;
+    s += cnt[k];
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = s;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = (lane < (int)(blockDim.x >> 5)) ? wsum[lane] : 0u;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    wsum[lane] = w;
+  }
+  __syncthreads();
+  uint32_t run = inc - s + (warp > 0 ? wsum[warp - 1] : 0u);
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k) {
+    if (b + k < n) {
+      run += cnt[k];
+      offsets[b + k + 1] = run;
+    }
+  }
+  if (threadIdx.x == 0) offsets[0] = 0u;
+  if (b < n && b + kScanPer >= n) {   // the thread that owns the last cell
+    h->total = (int32_t)run;
+    h->valid = ((int64_t)run <= (int64_t)h->capacity) ? 1 : 0;
+  }
+}
+
+__global__ void table_fill_kernel(const float *codebook, const SearchHeader *h, const uint32_t *offsets,
+                                  uint16_t *cand) {
+  const int lane = threadIdx.x & 31;
+  const int cell = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+  const SearchHeader hh = *h;
+  if (!hh.valid || cell >= hh.G * hh.G) return;
+  double x0, x1, y0, y1;
+  cell_bounds(hh, cell, x0, x1, y0, y1);
+  const double bound = cell_bound(codebook, hh.N, x0, x1, y0, y1, lane);
+  uint32_t pos = offsets[cell];
+  for (int base = 0; base < hh.N; base += 32) {
+    const int i = base + lane;
+    const bool keep = i < hh.N && dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
+    const uint32_t m = __ballot_sync(0xffffffffu, keep);
+    if (keep) cand[pos + __popc(m & ((1u << lane) - 1u))] = (uint16_t)i;
+    pos += __popc(m);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_build_search_table(const float *codebook, int N, void *table, cudaStream_t s) {
+  const int G = search_grid(N);
+  SearchHeader *h = reinterpret_cast<SearchHeader *>(table);
+  uint32_t *offsets = reinterpret_cast<uint32_t *>(reinterpret_cast<unsigned char *>(table) + sizeof(SearchHeader));
+  uint16_t *cand = reinterpret_cast<uint16_t *>(offsets + G * G + 1);
+  table_header_kernel<<<1, 1024, 0, s>>>(codebook, N, G, search_capacity(N), h);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int cells = G * G;
+  const int threads = 256;
+  const int blocks = (cells * 32 + threads - 1) / threads;
+  table_count_kernel<<<blocks, threads, 0, s>>>(codebook, h, offsets);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  table_scan_kernel<<<1, 1024, 0, s>>>(h, offsets);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  table_fill_kernel<<<blocks, threads, 0, s>>>(codebook, h, offsets, cand);
+  return cudaGetLastError();
+}
+
+}  // namespace qamw
