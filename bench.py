@@ -56,6 +56,8 @@ def parse_args(argv=None):
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
     p.add_argument("--search", choices=("pruned", "brute"), default="pruned",
                    help="nearest-centroid search: exact pruned table (default) or brute force")
+    p.add_argument("--brute-steps", type=int, default=3,
+                   help="extra brute-force encodes timed after the steps (FP32 roofline of that search)")
     return p.parse_args(argv)
 
 
@@ -220,6 +222,42 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------------------
+# work accounting of the pruned search (outside the timed region)
+# ---------------------------------------------------------------------------
+
+def pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec) -> int:
+    """Distance evaluations the exact pruned search performs on this matrix: for
+    every pair, the length of its grid cell's candidate list, or N for a pair
+    outside the grid. x is recomputed through the library's fp64 rotation hook
+    (qamw_rotate_rows) on U = w * s / r, in row blocks; the cell arithmetic is
+    the encode's fp32 one, on the table header's constants."""
+    import torch
+    raw = table[:48].cpu().numpy()
+    G = int(raw[8:12].view(np.int32)[0])
+    a, UL, inv = (float(v) for v in raw[24:36].view(np.float32))
+    nbytes_off = 4 * (G * G + 1)
+    offsets = table[48:48 + nbytes_off].view(torch.int32).to(torch.int64)
+    lens = (offsets[1:] - offsets[:-1])
+    M, K = Wd.shape
+    sig = sigma.to(torch.float64)
+    total = 0
+    for r0 in range(0, M, 1024):
+        r1 = min(M, r0 + 1024)
+        U = Wd[r0:r1].to(torch.float64) * cscale.to(torch.float64)[None, :]
+        rr = rnorm[r0:r1].to(torch.float64)[:, None]
+        U = torch.where(rr > 0, U / torch.where(rr > 0, rr, torch.ones_like(rr)), torch.zeros_like(U))
+        Y = q.rotate_rows(U.contiguous(), spec.block, spec.seed)
+        x = (Y.view(r1 - r0, K // 2, 2) / sig[None, :, None]).to(torch.float32)
+        u = x / (a + x.abs())
+        f = (u + UL) * inv
+        inside = (f >= 0).all(-1) & (f < G).all(-1)
+        cell = f[..., 1].clamp(0, G - 1).to(torch.int64) * G + f[..., 0].clamp(0, G - 1).to(torch.int64)
+        n = torch.where(inside, lens[cell], torch.full_like(cell, spec.N))
+        total += int(n.sum().item())
+    return total
 
 
 # ---------------------------------------------------------------------------
@@ -420,22 +458,59 @@ def run_ours(args):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     fp32_peak = sms * FP32_LANES_PER_SM * sm_max * 1e6  # FP32 lane-instructions per second
     P = M * K // 2
-    enc_ops = 4.0 * P * spec.N              # 2 sub + 1 mul + 1 fma per (pair, centroid)
     enc_ms = statistics.mean(t_enc)
     dec_ms = statistics.mean(t_dec)
     cal_ms = statistics.mean(t_cal)
     dec_bytes = M * K * 2 + M * wpr * 4 + 4 * M + 4 * K + 2 * K + 8 * spec.N
     cal_bytes = M * K * 2 * 2 + 4 * K + 4 * M
-    enc_roof = {"bound": "alu", "achieved": enc_ops / (enc_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
-                "unit": "Gop/s", "frac": enc_ops / (enc_ms * 1e-3) / fp32_peak, "traffic": None,
-                "kernel": "encode_kernel (brute-force search; events span the qamw_encode call)",
-                "peak_source": f"{sms} SMs x 128 FP32 lanes x {sm_max:.0f} MHz ({peak_kind} max clock)"}
+    fp32_src = f"{sms} SMs x 128 FP32 lanes x {sm_max:.0f} MHz ({peak_kind} max clock)"
+    # brute-force encode, timed on its own (not part of the step): its search is
+    # FP32-bound, 4 FP32 operations (2 FSUB, FMUL, FFMA) per pair and centroid
+    brute_ms = None
+    if args.search == "pruned" and args.brute_steps > 0:
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.brute_steps)]
+        q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sigma, Cd, spec.bits, status=status,
+                 out=(packed, rnorm, cscale))
+        for e0, e1 in bev:
+            flush.fill_(2.0)
+            e0.record(stream)
+            q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sigma, Cd, spec.bits, status=status,
+                     out=(packed, rnorm, cscale))
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        brute_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in bev)
+        # restore the pruned encoding (identical by construction) for e2e / checks
+        one()
+        torch.cuda.synchronize(dev)
+    elif args.search == "brute":
+        brute_ms = enc_ms
+    brute_roof = None
+    if brute_ms is not None:
+        ops = 4.0 * P * spec.N
+        brute_roof = {"bound": "alu", "achieved": ops / (brute_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
+                      "unit": "Gop/s", "frac": ops / (brute_ms * 1e-3) / fp32_peak, "traffic": None,
+                      "kernel": "encode_kernel (brute-force search; events span the qamw_encode call)",
+                      "ms": brute_ms, "peak_source": fp32_src}
+    if args.search == "pruned":
+        evals = pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec)
+        ops = 4.0 * evals
+        enc_roof = {"bound": "alu", "achieved": ops / (enc_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
+                    "unit": "Gop/s", "frac": ops / (enc_ms * 1e-3) / fp32_peak, "traffic": None,
+                    "kernel": "encode_pruned_kernel (exact pruned search; events span the qamw_encode call)",
+                    "evaluations_per_pair": evals / P, "peak_source": fp32_src,
+                    "hbm_gbs": (M * K * 2 + M * wpr * 4) / (enc_ms * 1e-3) / 1e9}
+    else:
+        enc_roof = brute_roof
     dec_roof = {"bound": "hbm", "achieved": dec_bytes / (dec_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": dec_bytes / (dec_ms * 1e-3) / 1e9 / hbm, "traffic": None, "kernel": "decode_kernel",
                 "peak_source": f"{peak_kind} hbm_gbs", "gweights_per_s": weights / (dec_ms * 1e-3) / 1e9}
     cal_roof = {"bound": "hbm", "achieved": cal_bytes / (cal_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": cal_bytes / (cal_ms * 1e-3) / 1e9 / hbm, "traffic": None,
                 "kernel": "qamw_calibrate_sigma (4 kernels)"}
+    rooflines = {"encode": enc_roof, "decode": dec_roof, "calibrate": cal_roof}
+    if brute_roof is not None:
+        rooflines["encode_brute_force"] = brute_roof
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -492,11 +567,12 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; no checkpoint)",
             "config": {"workload": wname, "M": M, "K": K, "weight_dtype": spec.dtype, "block": spec.block,
-                       "N": spec.N, "bits": spec.bits, "alpha": spec.alpha, "search": "brute-force",
+                       "N": spec.N, "bits": spec.bits, "alpha": spec.alpha,
+                       "search": "exact pruned (grid table)" if args.search == "pruned" else "brute force",
                        "l2": "flushed by a 256 MiB write before every timed step",
                        "parallelism": f"{world} independent replica(s)"},
             "roofline": enc_roof,
-            "rooflines": {"encode": enc_roof, "decode": dec_roof, "calibrate": cal_roof},
+            "rooflines": rooflines,
             "ms": {"calibrate": cal_ms, "encode": enc_ms, "decode": dec_ms},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 8 * args.steps, "clocks": clk,
             "dtype_detail": "rotation fp64, search and decode fp32, decode output bf16",

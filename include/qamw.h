@@ -66,7 +66,7 @@ enum {
 #define QAMW_STATUS_BAD_INDEX 1u        /* decode: an index >= N (decoded as 0) */
 #define QAMW_STATUS_NONFINITE_NORM 2u   /* a row norm is Inf/NaN */
 #define QAMW_STATUS_BAD_ACT_RMS 4u      /* an act_rms entry is not finite and > 0 */
-#define QAMW_STATUS_NONFINITE_INPUT 8u  /* a weight is Inf/NaN (its pairs coded as index 0) */
+#define QAMW_STATUS_NONFINITE_INPUT 8u  /* encode: a row norm is Inf/NaN (the row is coded as zero pairs) or a sigma_k gives no finite fp32 pair (1/sigma_k not finite or beyond the fp32 range) */
 #define QAMW_STATUS_TIMEOUT 16u         /* a bounded wait on an asynchronous copy ran out; output incomplete */
 
 /* Maximum sizes of this build. */
@@ -144,7 +144,7 @@ int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K
  * Errors: as qamw_calibrate_sigma (except EWORKSPACE), plus QAMW_EUNSUPPORTED
  * for shapes beyond the limit and QAMW_ECUDA if the address lookup fails.
  */
-#define QAMW_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define QAMW_NOALLOC_SCRATCH_BYTES (8u << 20)
 int qamw_calibrate_sigma_noalloc(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
                                  const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
                                  float *sigma_out, int32_t *status, qamw_stream_t stream);

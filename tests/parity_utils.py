@@ -29,8 +29,9 @@ def to_gpu_matrix(w32: np.ndarray, dtype: str):
     return torch.from_numpy(np.ascontiguousarray(w32)).cuda(), w32
 
 
-def gpu_codec(Wd, act, alpha, block, seed, C, bits, sigma=None):
-    """calibrate (unless sigma given) + encode on the GPU; returns numpy results."""
+def gpu_codec(Wd, act, alpha, block, seed, C, bits, sigma=None, search="brute"):
+    """calibrate (unless sigma given) + encode on the GPU; returns numpy results.
+    search: "brute" (no table) or "pruned" (the codebook's search table)."""
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     act_d = None if act is None else torch.from_numpy(act).cuda()
     if sigma is None:
@@ -38,7 +39,8 @@ def gpu_codec(Wd, act, alpha, block, seed, C, bits, sigma=None):
     else:
         sig_d = torch.from_numpy(sigma).cuda()
     Cd = torch.from_numpy(np.ascontiguousarray(C, dtype=np.float32)).cuda()
-    enc = qamw.encode(Wd, act_d, alpha, block, seed, sig_d, Cd, bits, status=status)
+    table = qamw.build_search_table(Cd) if search == "pruned" else None
+    enc = qamw.encode(Wd, act_d, alpha, block, seed, sig_d, Cd, bits, status=status, search_table=table)
     torch.cuda.synchronize()
     return {
         "sigma": sig_d.cpu().numpy(), "r": enc.row_norm.cpu().numpy(), "s": enc.col_scale.cpu().numpy(),

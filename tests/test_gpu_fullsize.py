@@ -35,7 +35,7 @@ def _check_encode(spec, n_rows=12):
     act = synth.act_for(spec)
     Wd, W = to_gpu_matrix(w32, spec.dtype)
     C = qamw.load_codebook(spec.N)
-    g = gpu_codec(Wd, act, spec.alpha, spec.block, spec.seed, C, spec.bits)
+    g = gpu_codec(Wd, act, spec.alpha, spec.block, spec.seed, C, spec.bits, search="pruned")
     assert g["status"] == 0
     sig = codec.calibrate_sigma(W, act, spec.alpha, spec.block, spec.seed)
     n_sig = int(np.sum(g["sigma"] != sig))

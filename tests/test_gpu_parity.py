@@ -74,15 +74,16 @@ ENC_CASES = [
 ]
 
 
+@pytest.mark.parametrize("search", ["brute", "pruned"])
 @pytest.mark.parametrize("M,K,b,N,bits,dtype,alpha", ENC_CASES)
-def test_encode_pipeline_parity(M, K, b, N, bits, dtype, alpha):
+def test_encode_pipeline_parity(M, K, b, N, bits, dtype, alpha, search):
     rng = np.random.default_rng(M * 7 + K)
     w32 = (rng.standard_normal((M, K)) * 0.02).astype(np.float32)
     act = np.exp(rng.standard_normal(K) * 1.0).astype(np.float32)
     Wd, W = to_gpu_matrix(w32, dtype)
     C = _codebook(N)
     seed = 1000 + M
-    g = gpu_codec(Wd, act, alpha, b, seed, C, bits)
+    g = gpu_codec(Wd, act, alpha, b, seed, C, bits, search=search)
     sig = codec.calibrate_sigma(W, act, alpha, b, seed)
     assert np.array_equal(g["sigma"], sig)
     assert g["status"] == 0
@@ -110,7 +111,7 @@ def test_encode_special_rows():
     W[7] = np.random.default_rng(1).standard_normal(K).astype(np.float32) * 1e-20
     C = _codebook(N)
     Wd = torch.from_numpy(W).cuda()
-    g = gpu_codec(Wd, None, 0.0, b, 5, C, bits)
+    g = gpu_codec(Wd, None, 0.0, b, 5, C, bits, search="pruned")
     sig = codec.calibrate_sigma(W, None, 0.0, b, 5)
     assert np.array_equal(g["sigma"], sig)
     enc = codec.encode(W, None, 0.0, b, 5, sig, C, bits)

@@ -20,16 +20,26 @@ def _built(lib):
     return lib
 
 
+HEADER_BYTES = 48
+
+
 def _read_table(table):
     raw = table.cpu().numpy()
-    hdr = raw[:32].view(np.int32)
-    magic, N, G, total = int(hdr[0]) & 0xFFFFFFFF, int(hdr[1]), int(hdr[2]), int(hdr[3])
-    L, inv = raw[16:24].view(np.float32)
-    valid = int(raw[24:28].view(np.int32)[0])
-    offsets = raw[32:32 + 4 * (G * G + 1)].view(np.uint32).astype(np.int64)
-    cand = raw[32 + 4 * (G * G + 1):].view(np.uint16)[:total].astype(np.int64)
-    return dict(magic=magic, N=N, G=G, total=total, L=float(L), inv=float(inv), valid=valid, offsets=offsets,
-                cand=cand)
+    hdr = raw[:HEADER_BYTES].view(np.int32)
+    magic, N, G, total, valid, cap = (int(hdr[0]) & 0xFFFFFFFF, int(hdr[1]), int(hdr[2]), int(hdr[3]),
+                                      int(hdr[4]), int(hdr[5]))
+    a, UL, inv, L = raw[24:40].view(np.float32)
+    offsets = raw[HEADER_BYTES:HEADER_BYTES + 4 * (G * G + 1)].view(np.uint32).astype(np.int64)
+    cand = raw[HEADER_BYTES + 4 * (G * G + 1):].view(np.uint16)[:total].astype(np.int64)
+    return dict(magic=magic, N=N, G=G, total=total, valid=valid, capacity=cap, a=np.float32(a),
+                UL=np.float32(UL), inv=np.float32(inv), L=float(L), offsets=offsets, cand=cand)
+
+
+def _cell_coord(x, t):
+    """The encode's fp32 cell coordinate: (x / (a + |x|) + UL) * inv_cw."""
+    x = x.astype(np.float32)
+    u = (x / (t["a"] + np.abs(x))).astype(np.float32)
+    return ((u + t["UL"]).astype(np.float32) * t["inv"]).astype(np.float32)
 
 
 @pytest.mark.parametrize("N", [4, 16, 128, 256, 1024, 2048])
@@ -38,23 +48,28 @@ def test_table_lists_the_nearest_centroid_of_every_point(N):
     t = _read_table(qamw.build_search_table(torch.from_numpy(C).cuda()))
     assert t["valid"] == 1 and t["N"] == N
     G, L, off, cand = t["G"], t["L"], t["offsets"], t["cand"]
+    assert L > np.abs(C).max()
     assert off[0] == 0 and off[-1] == t["total"] and np.all(np.diff(off) >= 1)
     for k in range(G * G):
         lst = cand[off[k]:off[k + 1]]
         assert np.all(np.diff(lst) > 0) and lst.max() < N
-    # random points, half of them within 1e-4 cells of a cell edge
+    # random points: a Gaussian cloud, a uniform spread over [-L, L]^2, and
+    # points within 1e-4 cells of a cell edge (edges mapped back to x)
     rng = np.random.default_rng(N)
-    pts = rng.uniform(-L, L, size=(200000, 2)).astype(np.float32)
-    edge = rng.integers(0, G + 1, size=(100000, 2)) * (2 * L / G) - L
-    pts[:100000] = (edge + rng.uniform(-1e-4, 1e-4, size=edge.shape) * (2 * L / G)).astype(np.float32)
-    fx = ((pts[:, 0] + np.float32(L)) * np.float32(t["inv"])).astype(np.float32)
-    fy = ((pts[:, 1] + np.float32(L)) * np.float32(t["inv"])).astype(np.float32)
+    a, UL, inv = float(t["a"]), float(t["UL"]), float(t["inv"])
+    edge_u = rng.integers(0, G + 1, size=(100000, 2)) / inv - UL
+    edge_u = edge_u + rng.uniform(-1e-4, 1e-4, size=edge_u.shape) / inv
+    edge_u = np.clip(edge_u, -0.999, 0.999)
+    edge_x = a * edge_u / (1.0 - np.abs(edge_u))
+    pts = np.concatenate([rng.standard_normal((100000, 2)), rng.uniform(-L, L, size=(100000, 2)),
+                          edge_x]).astype(np.float32)
+    fx, fy = _cell_coord(pts[:, 0], t), _cell_coord(pts[:, 1], t)
     inside = (fx >= 0) & (fx < G) & (fy >= 0) & (fy < G)
+    assert inside.mean() > 0.9
     cell = fy[inside].astype(np.int64) * G + fx[inside].astype(np.int64)
     idx, _ = codec.nearest_centroid(pts[inside], C)
     for c, i in zip(cell, idx):
-        lst = cand[off[c]:off[c + 1]]
-        assert i in lst
+        assert i in cand[off[c]:off[c + 1]]
 
 
 CASES = [
@@ -65,6 +80,9 @@ CASES = [
     (9, 96, 32, 16, 4, "f32"),
     (5, 24, 8, 4, 2, "f32"),
     (17, 1536, 512, 128, 7, "bf16"),
+    (6, 2048, 1024, 256, 8, "bf16"),     # b = 1024: the table is not used (brute-force kernel)
+    (300, 1000, 8, 1024, 10, "bf16"),    # K not a multiple of 16: a lane partly past K
+    (20, 1004, 4, 256, 8, "bf16"),       # rows not 16-byte aligned: scalar loads
 ]
 
 

@@ -66,16 +66,46 @@ __device__ __forceinline__ double load_w(const void *W, int64_t off) {
 }
 
 template <int WT>
-__global__ void __launch_bounds__(256) row_norm_kernel(RowNormArgs a) {
+__global__ void __launch_bounds__(256) row_norm_kernel(RowNormArgs a, int vec_ok) {
   const int lane = threadIdx.x & 31;
   const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  constexpr int kEpv = (WT == QAMW_BF16) ? 8 : 4;   // elements per 16-byte load
   for (int64_t row = gw; row < a.M; row += nw) {
     const int64_t base = row * a.ldw;
     double acc = 0.0;
-    for (int64_t j = lane; j < a.K; j += 32) {
-      const double v = load_w<WT>(a.W, base + j) * (double)a.s[j];
-      acc = fma(v, v, acc);
+    if (vec_ok) {   // K % kEpv == 0, W rows and s 16-byte aligned
+#pragma unroll 4
+      for (int64_t j = (int64_t)lane * kEpv; j < a.K; j += 32 * kEpv) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.W) +
+                                                              (base + j) * (WT == QAMW_BF16 ? 2 : 4)));
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        if (WT == QAMW_BF16) {
+          const float4 s0 = __ldg(reinterpret_cast<const float4 *>(a.s + j));
+          const float4 s1 = __ldg(reinterpret_cast<const float4 *>(a.s + j + 4));
+          const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const double v0 = bf16_bits_to_double(w4[h] & 0xffffu) * (double)sv[2 * h];
+            const double v1 = bf16_bits_to_double(w4[h] >> 16) * (double)sv[2 * h + 1];
+            acc = fma(v0, v0, acc);
+            acc = fma(v1, v1, acc);
+          }
+        } else {
+          const float4 s0 = __ldg(reinterpret_cast<const float4 *>(a.s + j));
+          const float sv[4] = {s0.x, s0.y, s0.z, s0.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const double v = (double)__uint_as_float(w4[h]) * (double)sv[h];
+            acc = fma(v, v, acc);
+          }
+        }
+      }
+    } else {
+      for (int64_t j = lane; j < a.K; j += 32) {
+        const double v = load_w<WT>(a.W, base + j) * (double)a.s[j];
+        acc = fma(v, v, acc);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -229,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate_kernel(CalibArgs a, int
       rotate_row_lane<WT>(v, ra, &tab.sd[lane * kSdPitch], row, col_lane, vec_ok != 0, lane);
       const double q = inv_sqrt_b / (double)r;
 #pragma unroll
-      for (int p = 0; p < 16; ++p) acc[p] += q * sqrt(v[2 * p] * v[2 * p] + v[2 * p + 1] * v[2 * p + 1]);
+      for (int p = 0; p < 16; ++p)
+        acc[p] += q * sqrt(__dadd_rn(__dmul_rn(v[2 * p], v[2 * p]), __dmul_rn(v[2 * p + 1], v[2 * p + 1])));
     }
     const int64_t pbase = col_lane >> 1;
 #pragma unroll
@@ -325,116 +356,20 @@ __device__ __forceinline__ void search_brute16(const float4 *__restrict__ cb4, i
   }
 }
 
-// Exact pruned search (table from qamw_search.cu, copied to shared memory):
-// the pair's grid cell lists every centroid that can be an fp32 minimiser;
-// the list is in ascending index order, so a strict "<" keeps the lowest index
-// among equal distances -- the brute-force result. A pair outside the grid
-// (or not finite) scans the whole codebook.
-__device__ __forceinline__ void search_pruned16(const float2 *__restrict__ cb2, int n_all,
-                                                const uint16_t *__restrict__ toff,
-                                                const uint16_t *__restrict__ cand, int G, float L, float inv_cw,
-                                                const float (&x0)[16], const float (&x1)[16], int (&out)[16]) {
-  // cell ranges of all 16 pairs first (independent loads)
-  int beg[16], end[16];
-#pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    const float fx = __fmul_rn(__fadd_rn(x0[p], L), inv_cw);
-    const float fy = __fmul_rn(__fadd_rn(x1[p], L), inv_cw);
-    if (fx >= 0.0f && fx < (float)G && fy >= 0.0f && fy < (float)G) {
-      const int cell = (int)fy * G + (int)fx;
-      beg[p] = toff[cell];
-      end[p] = toff[cell + 1];
-    } else {
-      beg[p] = -1;   // outside the grid: every centroid
-      end[p] = n_all;
-    }
-  }
-#pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    float best = INFINITY;
-    int bi = 0;
-    if (beg[p] >= 0) {
-      int j = beg[p];
-      const int e = end[p];
-      for (; j + 4 <= e; j += 4) {
-        const int i0 = cand[j], i1 = cand[j + 1], i2 = cand[j + 2], i3 = cand[j + 3];
-        const float2 c0 = cb2[i0], c1 = cb2[i1], c2 = cb2[i2], c3 = cb2[i3];
-        const float d0 = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
-        const float d1 = dist2_scalar(x0[p], x1[p], c1.x, c1.y);
-        const float d2 = dist2_scalar(x0[p], x1[p], c2.x, c2.y);
-        const float d3 = dist2_scalar(x0[p], x1[p], c3.x, c3.y);
-        if (d0 < best) { best = d0; bi = i0; }
-        if (d1 < best) { best = d1; bi = i1; }
-        if (d2 < best) { best = d2; bi = i2; }
-        if (d3 < best) { best = d3; bi = i3; }
-      }
-      for (; j < e; ++j) {
-        const int i0 = cand[j];
-        const float2 c0 = cb2[i0];
-        const float d0 = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
-        if (d0 < best) { best = d0; bi = i0; }
-      }
-    } else {
-      for (int i0 = 0; i0 < end[p]; ++i0) {
-        const float2 c0 = cb2[i0];
-        const float d0 = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
-        if (d0 < best) { best = d0; bi = i0; }
-      }
-    }
-    out[p] = bi;
-  }
-}
-
-template <int WT, int CHUNK, bool PRUNED>
-__global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeArgs a, int vec_ok, int tab_cap) {
+template <int WT, int CHUNK>
+__global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeArgs a, int vec_ok) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_pad = (a.N + CHUNK - 1) / CHUNK * CHUNK;
-  // brute force: (c0, c0, c1, c1) per centroid for the packed pipeline; pruned:
-  // (c0, c1), which halves the bank traffic of its per-lane gathers
-  constexpr size_t kCbEntry = PRUNED ? sizeof(float2) : sizeof(float4);
+  // (c0, c0, c1, c1) per centroid for the packed fp32x2 pipeline
   float4 *cb4 = reinterpret_cast<float4 *>(smem_raw);
-  float2 *cb2 = reinterpret_cast<float2 *>(smem_raw);
-  WarpTables &tab = reinterpret_cast<WarpTables *>(smem_raw + (size_t)n_pad * kCbEntry)[warp];
+  WarpTables &tab = reinterpret_cast<WarpTables *>(smem_raw + (size_t)n_pad * sizeof(float4))[warp];
   for (int c = threadIdx.x; c < n_pad; c += blockDim.x) {
     float c0 = kFarCentroid, c1 = kFarCentroid;
     if (c < a.N) { c0 = a.codebook[2 * c]; c1 = a.codebook[2 * c + 1]; }
-    if constexpr (PRUNED) cb2[c] = make_float2(c0, c1);
-    else cb4[c] = make_float4(c0, c0, c1, c1);
-  }
-  // search table -> shared memory as 16-bit offsets and indices (if it fits)
-  __shared__ int s_use, s_G;
-  __shared__ float s_L, s_inv;
-  uint16_t *toff = reinterpret_cast<uint16_t *>(smem_raw + (size_t)n_pad * kCbEntry + sizeof(WarpTables) * kWarps);
-  uint16_t *tcand = nullptr;
-  if constexpr (PRUNED) {
-    const SearchHeader *h = reinterpret_cast<const SearchHeader *>(a.table);
-    if (threadIdx.x == 0) {
-      const SearchHeader hh = *h;
-      const int cells = hh.G * hh.G;
-      const bool ok = hh.magic == kSearchMagic && hh.valid && hh.N == a.N && hh.G >= 1 && hh.G <= 128 &&
-                      hh.total >= 0 && hh.total <= tab_cap && hh.total < 65536;
-      s_use = ok ? 1 : 0;
-      s_G = hh.G;
-      s_L = hh.L;
-      s_inv = hh.inv_cw;
-      (void)cells;
-    }
-    __syncthreads();
-    if (s_use) {
-      const int cells = s_G * s_G;
-      const uint32_t *goff = reinterpret_cast<const uint32_t *>(reinterpret_cast<const unsigned char *>(a.table) +
-                                                                sizeof(SearchHeader));
-      const uint16_t *gcand = reinterpret_cast<const uint16_t *>(goff + cells + 1);
-      tcand = toff + ((cells + 1 + 7) & ~7);
-      const int total = (int)goff[cells];
-      for (int i = threadIdx.x; i <= cells; i += blockDim.x) toff[i] = (uint16_t)goff[i];
-      for (int i = threadIdx.x; i < total; i += blockDim.x) tcand[i] = gcand[i];
-    }
+    cb4[c] = make_float4(c0, c0, c1, c1);
   }
   __syncthreads();
-  const bool use_table = PRUNED && s_use;
-  if (PRUNED && s_use) tcand = toff + ((s_G * s_G + 1 + 7) & ~7);
 
   const RotateArgs &ra = a.rot;
   const int64_t n_chunks = (ra.K + kUnitCols - 1) / kUnitCols;
@@ -475,14 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeArgs a, int v
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
     int idx[16];
-    if constexpr (PRUNED) {
-      if (use_table)
-        search_pruned16(cb2, n_pad, toff, tcand, s_G, s_L, s_inv, x0, x1, idx);
-      else
-        search_pruned16(cb2, n_pad, toff, tcand, 0, 0.0f, 0.0f, x0, x1, idx);   // G = 0: every pair scans all
-    } else {
-      search_brute16<CHUNK>(cb4, n_pad, x0, x1, idx);
-    }
+    search_brute16<CHUNK>(cb4, n_pad, x0, x1, idx);
     // pack: stage the unit's 512 indices, then build the unit's words
     __syncwarp();
 #pragma unroll
@@ -560,69 +488,61 @@ cudaError_t launch_channel_scale(const ScaleArgs &a, cudaStream_t s) {
 cudaError_t launch_row_norms(const RowNormArgs &a, cudaStream_t s) {
   const int threads = 256;
   const int64_t blocks = std::min<int64_t>((a.M + 7) / 8, (int64_t)sm_count() * 8);
+  const int epv = (a.wt == QAMW_BF16) ? 8 : 4;
+  const int vec = (w_vec_ok(a.W, a.wt, a.ldw) && a.K % epv == 0 && reinterpret_cast<uintptr_t>(a.s) % 16 == 0) ? 1 : 0;
   if (a.wt == QAMW_BF16)
-    row_norm_kernel<QAMW_BF16><<<(int)blocks, threads, 0, s>>>(a);
+    row_norm_kernel<QAMW_BF16><<<(int)blocks, threads, 0, s>>>(a, vec);
   else
-    row_norm_kernel<QAMW_F32><<<(int)blocks, threads, 0, s>>>(a);
+    row_norm_kernel<QAMW_F32><<<(int)blocks, threads, 0, s>>>(a, vec);
   return cudaGetLastError();
 }
 
 cudaError_t launch_calibrate(const CalibArgs &a, cudaStream_t s) {
-  const size_t smem = sizeof(WarpTables) * kWarps;
-  const int64_t n_chunks = (a.rot.K + kUnitCols - 1) / kUnitCols;
-  const int64_t units = n_chunks * a.groups;
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((units + kWarps - 1) / kWarps, sm_count()));
-  const int vec = w_vec_ok(a.rot.W, a.rot.wt, a.rot.ldw) ? 1 : 0;
   cudaError_t e;
-  if (a.rot.wt == QAMW_BF16) {
-    if ((e = set_smem(calibrate_kernel<QAMW_BF16>, smem)) != cudaSuccess) return e;
-    calibrate_kernel<QAMW_BF16><<<(int)blocks, kThreads, smem, s>>>(a, vec);
+  if (a.rot.log2b <= 9) {
+    if ((e = launch_calibrate_partials512(a, s)) != cudaSuccess) return e;
   } else {
-    if ((e = set_smem(calibrate_kernel<QAMW_F32>, smem)) != cudaSuccess) return e;
-    calibrate_kernel<QAMW_F32><<<(int)blocks, kThreads, smem, s>>>(a, vec);
+    const size_t smem = sizeof(WarpTables) * kWarps;
+    const int64_t n_chunks = (a.rot.K + kUnitCols - 1) / kUnitCols;
+    const int64_t units = n_chunks * a.groups;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((units + kWarps - 1) / kWarps, sm_count()));
+    const int vec = w_vec_ok(a.rot.W, a.rot.wt, a.rot.ldw) ? 1 : 0;
+    if (a.rot.wt == QAMW_BF16) {
+      if ((e = set_smem(calibrate_kernel<QAMW_BF16>, smem)) != cudaSuccess) return e;
+      calibrate_kernel<QAMW_BF16><<<(int)blocks, kThreads, smem, s>>>(a, vec);
+    } else {
+      if ((e = set_smem(calibrate_kernel<QAMW_F32>, smem)) != cudaSuccess) return e;
+      calibrate_kernel<QAMW_F32><<<(int)blocks, kThreads, smem, s>>>(a, vec);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t P = a.rot.K >> 1;
   sigma_reduce_kernel<<<(int)((P + 31) / 32), kReduceWarps * 32, 0, s>>>(a.partials, a.groups, P, a.rot.M,
                                                                           a.sigma_out);
   return cudaGetLastError();
 }
 
-template <int WT, int CHUNK, bool PRUNED>
+template <int WT, int CHUNK>
 static cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
   const int n_pad = (a.N + CHUNK - 1) / CHUNK * CHUNK;
-  size_t smem = (size_t)n_pad * (PRUNED ? sizeof(float2) : sizeof(float4)) + sizeof(WarpTables) * kWarps;
-  int tab_cap = 0;
-  if (PRUNED) {
-    int dev = 0, smem_max = 0;
-    cudaGetDevice(&dev);
-    cudaError_t e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e != cudaSuccess) return e;
-    const int G = search_grid(a.N);
-    const size_t off_bytes = (size_t)((G * G + 1 + 7) & ~7) * 2;
-    const int64_t room = ((int64_t)smem_max - 64 /*static*/ - (int64_t)smem - (int64_t)off_bytes) / 2;
-    tab_cap = (int)std::max<int64_t>(0, std::min<int64_t>(std::min<int64_t>(room, 65535), search_capacity(a.N)));
-    tab_cap &= ~7;
-    smem += off_bytes + (size_t)tab_cap * 2;
-  }
-  cudaError_t e = set_smem(encode_kernel<WT, CHUNK, PRUNED>, smem);
+  const size_t smem = (size_t)n_pad * sizeof(float4) + sizeof(WarpTables) * kWarps;
+  cudaError_t e = set_smem(encode_kernel<WT, CHUNK>, smem);
   if (e != cudaSuccess) return e;
   const int64_t n_chunks = (a.rot.K + kUnitCols - 1) / kUnitCols;
   const int64_t units = n_chunks * a.rot.M;
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((units + kWarps - 1) / kWarps, sm_count()));
   const int vec = w_vec_ok(a.rot.W, a.rot.wt, a.rot.ldw) ? 1 : 0;
-  encode_kernel<WT, CHUNK, PRUNED><<<(int)blocks, kThreads, smem, s>>>(a, vec, tab_cap);
+  encode_kernel<WT, CHUNK><<<(int)blocks, kThreads, smem, s>>>(a, vec);
   return cudaGetLastError();
 }
 
 template <int WT>
 static cudaError_t launch_encode_wt(const EncodeArgs &a, cudaStream_t s) {
-  const bool big = a.N >= 512;
-  if (a.table != nullptr) return big ? launch_encode_t<WT, 32, true>(a, s) : launch_encode_t<WT, 8, true>(a, s);
-  return big ? launch_encode_t<WT, 32, false>(a, s) : launch_encode_t<WT, 8, false>(a, s);
+  return (a.N >= 512) ? launch_encode_t<WT, 32>(a, s) : launch_encode_t<WT, 8>(a, s);
 }
 
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s) {
+  if (encode_pruned_applicable(a)) return launch_encode_pruned(a, s);
   return (a.rot.wt == QAMW_BF16) ? launch_encode_wt<QAMW_BF16>(a, s) : launch_encode_wt<QAMW_F32>(a, s);
 }
 

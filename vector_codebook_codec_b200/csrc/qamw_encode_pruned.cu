@@ -1,0 +1,264 @@
+// qamw_encode_pruned.cu -- QAM-W encode with the exact pruned
+// nearest-centroid search, for Hadamard blocks b <= 512.
+//
+// Method: "QAM-W: Joint 2D Codebook Quantization for LLM Weights via Hadamard
+// Rotation and Activation-Aware Scaling", Technical Summary, "Methodology:
+// The QAM-W Codec": normalise by the stored row norm (step 1), sign-masked
+// block Hadamard rotation (step 2), x = z / sigma (step 3), nearest centroid
+// (step 4) with the channel scale s_j applied first (step 5), then bit packing.
+//
+// Work decomposition. A *unit* is one row x 512 consecutive columns handled by
+// one warp: lane l owns columns [16l, 16l + 16) of the unit (8 pairs); the
+// rotation is the fp64 one of qamw_rotate16.cuh, which gives the same x bit
+// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 16 warps takes a contiguous
+// range of *tiles* (16 rows x one 512-column chunk) in chunk-major order; the
+// chunk's d_j * s_j and 1 / sigma_k live once per CTA in shared memory, next
+// to the codebook and the search table. The next unit's weights are loaded
+// while the current one is searched.
+//
+// Search. The pair's cell of the search table (qamw_search.cu) lists every
+// centroid that can be an fp32 minimiser, in ascending index order; a strict
+// "<" over the list keeps the lowest index among equal distances, which is the
+// brute-force result. In shared memory the lists follow an identity list
+// 0..N-1, which a pair outside the grid (or every pair, if the table does not
+// fit or does not match the codebook) scans instead.
+#include <algorithm>
+#include <cfloat>
+#include <cmath>
+
+#include "qamw_device.cuh"
+#include "qamw_internal.h"
+#include "qamw_rotate16.cuh"
+
+namespace qamw {
+namespace {
+
+constexpr int kWarps = kTileRows;
+constexpr int kThreads = kWarps * 32;
+
+struct ChunkTables {
+  double sd[32 * kSdPitch];       // d_j * s_j of the lane's 16 columns (0 past K)
+  double inv_sigma[32 * kIsPitch];  // 1 / sigma_k of the lane's 8 pairs (0 past K/2)
+};
+constexpr int kStageBytes = 512;  // per warp: 256 uint16 indices of the unit
+
+template <int WT>
+__global__ void __launch_bounds__(kThreads, 1)
+    encode_pruned_kernel(EncodeArgs a, int vec_ok, int tab_cap, int toff_slots) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const RotateArgs &ra = a.rot;
+  const int N = a.N;
+  const int n2 = (N + 1) & ~1;
+  ChunkTables &ct = *reinterpret_cast<ChunkTables *>(smem);
+  uint16_t *stage = reinterpret_cast<uint16_t *>(smem + sizeof(ChunkTables) + warp * kStageBytes);
+  float2 *cb2 = reinterpret_cast<float2 *>(smem + sizeof(ChunkTables) + kWarps * kStageBytes);
+  uint16_t *toff = reinterpret_cast<uint16_t *>(cb2 + n2);
+  uint16_t *lst = toff + toff_slots;   // identity list 0..N-1, then the cell lists
+
+  __shared__ int s_use, s_G;
+  __shared__ float s_a, s_UL, s_inv;
+  if (threadIdx.x == 0) {
+    const SearchHeader h = *reinterpret_cast<const SearchHeader *>(a.table);
+    const bool ok = h.magic == kSearchMagic && h.valid == 1 && h.N == N && h.G >= 1 && h.G <= 128 &&
+                    h.G * h.G + 1 <= toff_slots && h.total >= 0 && h.total <= tab_cap - N &&
+                    h.total + N < 65536 && h.a > 0.0f && h.UL > 0.0f && h.UL < 1.0f && h.inv_cw > 0.0f;
+    s_use = ok ? 1 : 0;
+    s_G = h.G;
+    s_a = h.a;
+    s_UL = h.UL;
+    s_inv = h.inv_cw;
+  }
+  for (int c = threadIdx.x; c < n2; c += kThreads)
+    cb2[c] = (c < N) ? make_float2(a.codebook[2 * c], a.codebook[2 * c + 1]) : make_float2(0.0f, 0.0f);
+  for (int i = threadIdx.x; i < N; i += kThreads) lst[i] = (uint16_t)i;
+  __syncthreads();
+  const bool use = s_use != 0;
+  const int G = s_G;
+  if (use) {
+    const uint32_t *goff = reinterpret_cast<const uint32_t *>(reinterpret_cast<const unsigned char *>(a.table) +
+                                                              sizeof(SearchHeader));
+    const uint16_t *gcand = reinterpret_cast<const uint16_t *>(goff + G * G + 1);
+    // clamped on the copy, so that no table content can index outside the
+    // lists or the codebook
+    const uint32_t total = goff[G * G] < (uint32_t)(tab_cap - N) ? goff[G * G] : (uint32_t)(tab_cap - N);
+    for (int i = threadIdx.x; i <= G * G; i += kThreads)
+      toff[i] = (uint16_t)((goff[i] < total ? goff[i] : total) + (uint32_t)N);
+    for (int i = threadIdx.x; i < (int)total; i += kThreads)
+      lst[N + i] = (gcand[i] < (uint16_t)N) ? gcand[i] : (uint16_t)(N - 1);
+  }
+  const float a_ax = s_a, UL = s_UL, inv_cw = s_inv, Gf = (float)G;
+
+  const int64_t M = ra.M, K = ra.K, P = K >> 1;
+  const int64_t n_chunks = (K + kUnit - 1) / kUnit;
+  const int64_t RG = (M + kTileRows - 1) / kTileRows;
+  const int64_t T = n_chunks * RG;
+  const int64_t t0 = (int64_t)blockIdx.x * T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
+  const double inv_sqrt_b = 1.0 / sqrt((double)(1 << ra.log2b));
+  const int B = a.bits;
+
+  // the next unit's weights and row norm, loaded while the current one is searched
+  auto prefetch = [&](int64_t t, WRegs<WT> &w, float &rn) -> bool {
+    const int64_t chunk = t / RG, row = (t % RG) * kTileRows + warp;
+    rn = 0.0f;
+    if (row >= M) return false;
+    rn = ra.r[row];
+    return load_unit16<WT>(w, ra.W, ra.ldw, K, row, chunk * kUnit + 16 * lane, vec_ok);
+  };
+
+  WRegs<WT> wn;
+  float rn_next = 0.0f;
+  bool full_next = (t0 < t1) ? prefetch(t0, wn, rn_next) : false;
+  int64_t cur_chunk = -1;
+  for (int64_t t = t0; t < t1; ++t) {
+    const int64_t chunk = t / RG, g = t % RG;
+    if (chunk != cur_chunk) {
+      __syncthreads();   // every warp is done with the previous chunk's tables (and the table copy is complete)
+      load_sd512(ct.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
+      if (threadIdx.x < kUnit / 2) {
+        // a rotated unit row has |y_j| <= 1 (to within the fp32 rounding of r),
+        // so |x| <= 1 / sigma_k: every x of the column is a finite fp32 when
+        // 1 / sigma_k is at most half the fp32 range (else the status says so)
+        const int i = threadIdx.x;
+        const int64_t p = chunk * (kUnit / 2) + i;
+        const double is = (p < P) ? 1.0 / (double)a.sigma[p] : 0.0;
+        ct.inv_sigma[(i >> 3) * kIsPitch + (i & 7)] = is;
+        if (!(fabs(is) <= 0.5 * (double)FLT_MAX)) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
+      }
+      __syncthreads();
+      cur_chunk = chunk;
+    }
+    const WRegs<WT> wc = wn;
+    const bool full = full_next;
+    const float r = rn_next;
+    if (t + 1 < t1) full_next = prefetch(t + 1, wn, rn_next);
+
+    const int64_t row = g * kTileRows + warp;
+    if (row >= M) continue;
+    const int64_t col = chunk * kUnit + 16 * lane;
+
+    float x0[8], x1[8];
+    uint32_t bad = 0;
+    if (r > 0.0f && isfinite(r)) {
+      double v[16];
+      scaled16<WT>(v, wc, full, ra.W, ra.ldw, K, row, col, &ct.sd[lane * kSdPitch]);
+      fwht16_fp64(v, ra.log2b, lane);
+      const double qn = inv_sqrt_b / (double)r;
+      const double2 *is2 = reinterpret_cast<const double2 *>(&ct.inv_sigma[lane * kIsPitch]);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const double2 is = is2[h];
+        const double f0 = qn * is.x, f1 = qn * is.y;
+        x0[2 * h] = (float)(v[4 * h] * f0);
+        x1[2 * h] = (float)(v[4 * h + 1] * f0);
+        x0[2 * h + 1] = (float)(v[4 * h + 2] * f1);
+        x1[2 * h + 1] = (float)(v[4 * h + 3] * f1);
+      }
+    } else {
+      if (!(r == 0.0f)) bad = 1;   // NaN / Inf row norm; a zero row codes every pair as x = 0
+#pragma unroll
+      for (int p = 0; p < 8; ++p) { x0[p] = 0.0f; x1[p] = 0.0f; }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
+
+    // candidate ranges of the 8 pairs (cell lists, or the identity list)
+    int beg[8], end[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      beg[p] = 0;
+      end[p] = N;
+      if (use) {
+        const float u0 = __fdividef(x0[p], __fadd_rn(a_ax, fabsf(x0[p])));
+        const float u1 = __fdividef(x1[p], __fadd_rn(a_ax, fabsf(x1[p])));
+        const float fx = __fmul_rn(__fadd_rn(u0, UL), inv_cw);
+        const float fy = __fmul_rn(__fadd_rn(u1, UL), inv_cw);
+        if (fx >= 0.0f && fx < Gf && fy >= 0.0f && fy < Gf) {
+          const int cell = (int)fy * G + (int)fx;
+          beg[p] = toff[cell];
+          end[p] = toff[cell + 1];
+        }
+      }
+    }
+    int idx[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      float best = INFINITY;
+      int bi = 0;
+      int j = beg[p];
+      const int e = end[p];
+      for (; j < e; ++j) {
+        const int i0 = lst[j];
+        const float2 c0 = cb2[i0];
+        const float d0 = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
+        if (d0 < best) { best = d0; bi = i0; }
+      }
+      idx[p] = bi;
+    }
+
+    // pack: stage the unit's 256 indices, then build the unit's words
+    __syncwarp();
+    reinterpret_cast<uint4 *>(stage)[lane] =
+        make_uint4((uint32_t)idx[0] | ((uint32_t)idx[1] << 16), (uint32_t)idx[2] | ((uint32_t)idx[3] << 16),
+                   (uint32_t)idx[4] | ((uint32_t)idx[5] << 16), (uint32_t)idx[6] | ((uint32_t)idx[7] << 16));
+    __syncwarp();
+    const int64_t pair0 = chunk * (kUnit / 2);
+    const int np = (int)((P - pair0) < (kUnit / 2) ? (P - pair0) : (kUnit / 2));
+    const int nw = (np * B + 31) >> 5;
+    uint32_t *dst = a.packed + row * a.wpr + chunk * (int64_t)(8 * B);
+    for (int w = lane; w < nw; w += 32) {
+      const int bit0 = w * 32;
+      const int k0 = bit0 / B;
+      const int k1 = min((bit0 + 31) / B, np - 1);
+      uint32_t word = 0;
+      for (int k = k0; k <= k1; ++k) {
+        const int off = k * B - bit0;
+        const uint32_t iv = stage[k];
+        word |= (off >= 0) ? (iv << off) : (iv >> (-off));
+      }
+      dst[w] = word;
+    }
+  }
+}
+
+template <typename Kern>
+cudaError_t set_smem(Kern k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int WT>
+cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
+  int dev = 0, smem_max = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  const int G = search_grid(a.N);
+  const int toff_slots = (G * G + 1 + 7) & ~7;
+  const int n2 = (a.N + 1) & ~1;
+  const size_t base = sizeof(ChunkTables) + (size_t)kWarps * kStageBytes + (size_t)n2 * sizeof(float2) +
+                      (size_t)toff_slots * 2;
+  const int64_t room = ((int64_t)smem_max - 128 /*static*/ - (int64_t)base) / 2;
+  int tab_cap = (int)std::max<int64_t>(0, std::min<int64_t>(room, 65535));
+  tab_cap &= ~7;
+  if (tab_cap < a.N) return cudaErrorInvalidConfiguration;   // the launcher only comes here for N <= 2048
+  const size_t smem = base + (size_t)tab_cap * 2;
+  if ((e = set_smem(encode_pruned_kernel<WT>, smem)) != cudaSuccess) return e;
+  const int64_t n_chunks = (a.rot.K + kUnit - 1) / kUnit;
+  const int64_t tiles = n_chunks * ((a.rot.M + kTileRows - 1) / kTileRows);
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count()));
+  const size_t es = (WT == QAMW_BF16) ? 2 : 4;
+  const int vec = ((reinterpret_cast<uintptr_t>(a.rot.W) % 16) == 0 && (a.rot.ldw * (int64_t)es) % 16 == 0) ? 1 : 0;
+  encode_pruned_kernel<WT><<<(int)blocks, kThreads, smem, s>>>(a, vec, tab_cap, toff_slots);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool encode_pruned_applicable(const EncodeArgs &a) {
+  return a.table != nullptr && a.rot.log2b <= 9 && a.N <= kPrunedMaxN;
+}
+
+cudaError_t launch_encode_pruned(const EncodeArgs &a, cudaStream_t s) {
+  return (a.rot.wt == QAMW_BF16) ? launch_t<QAMW_BF16>(a, s) : launch_t<QAMW_F32>(a, s);
+}
+
+}  // namespace qamw

@@ -12,19 +12,22 @@ namespace qamw {
 
 // Rows per calibration row group (fixed, so the fp64 reduction order -- and
 // hence sigma -- does not depend on the device or the grid size).
-constexpr int kCalibRowGroup = 4;
+constexpr int kCalibRowGroup = 16;
 // Columns handled by one warp in the encode / calibrate kernels (32 lanes x 32).
 constexpr int kUnitCols = 1024;
 
 // Header of a search table (see qamw_search.cu).
-constexpr uint32_t kSearchMagic = 0x54574D51u;   // "QMWT"
+constexpr uint32_t kSearchMagic = 0x32574D51u;   // "QMW2": table layout version 2
 struct SearchHeader {
   uint32_t magic;
   int32_t N, G, total;
-  float L, inv_cw;   // grid covers [-L, L]^2; cell index = floor((x + L) * inv_cw)
   int32_t valid, capacity;
+  // The grid is uniform in u = T(x) = x / (a + |x|) on each axis: cell index
+  // floor((T(x) + UL) * inv_cw), UL = T(L); it covers [-L, L]^2 in x.
+  float a, UL, inv_cw, L;
+  int32_t pad[2];
 };
-static_assert(sizeof(SearchHeader) == 32, "search header is 32 bytes");
+static_assert(sizeof(SearchHeader) == 48, "search header is 48 bytes");
 int search_grid(int N);
 int64_t search_capacity(int N);
 size_t search_table_bytes(int N);
@@ -107,7 +110,15 @@ struct RotateTestArgs {
 cudaError_t launch_channel_scale(const ScaleArgs &a, cudaStream_t s);
 cudaError_t launch_row_norms(const RowNormArgs &a, cudaStream_t s);
 cudaError_t launch_calibrate(const CalibArgs &a, cudaStream_t s);
+// The partial sums of the calibration for b <= 512 (qamw_calibrate.cu).
+cudaError_t launch_calibrate_partials512(const CalibArgs &a, cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+// Encode with the pruned search (qamw_encode_pruned.cu): a table given,
+// b <= 512 and N <= kPrunedMaxN; otherwise launch_encode takes the brute-force
+// kernel.
+constexpr int kPrunedMaxN = 2048;
+bool encode_pruned_applicable(const EncodeArgs &a);
+cudaError_t launch_encode_pruned(const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 // bf16 decode with TMA tensor loads/stores (qamw_decode_tma.cu).
 bool decode_tma_applicable(const DecodeArgs &a);

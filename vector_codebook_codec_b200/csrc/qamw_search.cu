@@ -3,9 +3,13 @@
 // Methodology (4) Joint 2D Quantization of the QAM-W page maps each normalised
 // pair x to the nearest centroid of one 2D codebook. The brute-force search
 // computes N distances per pair. This table lets the encode compute only the
-// distances that can matter: x-space is cut into a G x G grid of cells over
-// [-L, L]^2 (L a little beyond the outermost centroid); for every cell Q
-// (enlarged by a small margin) the table lists every centroid c with
+// distances that can matter. Each axis is mapped by the monotone
+// T(x) = x / (a + |x|), and the square [-L, L]^2 (L well beyond the outermost
+// centroid) is cut into G x G cells uniform in (T(x0), T(x1)): the cells are
+// small near the origin, where the pairs (unit circular Gaussian after the
+// sigma normalisation) and the centroids are dense, and grow outwards. For
+// every cell Q (enlarged by a small margin) the table lists every centroid c
+// with
 //     dmin(c, Q)^2 <= (1 + 1e-5) * D(Q)^2,   D(Q) = min_c' dmax(c', Q),
 // dmin / dmax being the least / greatest distance from c to a point of Q.
 // For a pair x in Q its exact nearest distance d* is at most D(Q), and every
@@ -15,6 +19,11 @@
 // "<" therefore returns exactly the index of the brute-force search (the
 // lowest index among the fp32 minimisers). Pairs outside the grid, or a table
 // that does not fit, use the brute-force search.
+//
+// The encode computes a pair's cell in fp32 as floor((T(x) + UL) * inv_cw)
+// with UL, inv_cw and a read from the header; its rounding error is below
+// 1e-4 of a cell, and the margin of 1e-3 cells that every cell is enlarged
+// by (in u, then mapped back to x in fp64) covers it.
 //
 // Table layout (device memory owned by the caller, 16-byte aligned):
 //   SearchHeader | uint32 offsets[G*G + 1] | uint16 cand[capacity]
@@ -29,7 +38,7 @@
 
 namespace qamw {
 
-int search_grid(int N) { return N >= 1024 ? 128 : (N >= 128 ? 64 : 32); }
+int search_grid(int N) { return N >= 64 ? 128 : 32; }
 
 int64_t search_capacity(int N) {
   const int G = search_grid(N);
@@ -46,6 +55,7 @@ namespace {
 
 constexpr double kCellMargin = 1e-3;   // cell enlargement, in cells (covers fp32 rounding of the cell index)
 constexpr double kTieSlack = 1e-5;     // relative slack on D(Q)^2
+constexpr float kAxisA = 2.0f;         // T(x) = x / (a + |x|): cells about 1/4 as wide at 0 as near |x| = 2
 
 __global__ void table_header_kernel(const float *codebook, int N, int G, int64_t capacity, SearchHeader *h) {
   __shared__ float red[32];
@@ -57,27 +67,37 @@ __global__ void table_header_kernel(const float *codebook, int N, int G, int64_t
   if (threadIdx.x == 0) {
     float r = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
-    const float L = r * 1.02f + 0.6f;
+    const float L = r * 1.5f + 2.0f;
+    const float UL = L / (kAxisA + L);
     h->magic = kSearchMagic;
     h->N = N;
     h->G = G;
     h->total = 0;
+    h->a = kAxisA;
+    h->UL = UL;
+    h->inv_cw = (float)G / (2.0f * UL);
     h->L = L;
-    h->inv_cw = (float)G / (2.0f * L);
+    h->pad[0] = h->pad[1] = 0;
     h->valid = 0;
     h->capacity = (int32_t)capacity;
   }
 }
 
-// Enlarged bounds of cell (ix, iy) in fp64.
+// Enlarged bounds of cell (ix, iy) in x, in fp64: the u-interval
+// [k / inv_cw - UL, (k + 1) / inv_cw - UL] widened by the margin, mapped back
+// through T^-1(u) = a u / (1 - |u|), and widened by a relative 1e-12 for the
+// fp64 rounding of that map.
+__device__ __forceinline__ double axis_inv(double a, double u) { return a * u / (1.0 - fabs(u)); }
 __device__ __forceinline__ void cell_bounds(const SearchHeader &h, int cell, double &x0, double &x1, double &y0,
                                             double &y1) {
   const int ix = cell % h.G, iy = cell / h.G;
-  const double L = (double)h.L, cw = 2.0 * L / (double)h.G, m = kCellMargin * cw;
-  x0 = -L + ix * cw - m;
-  x1 = -L + (ix + 1) * cw + m;
-  y0 = -L + iy * cw - m;
-  y1 = -L + (iy + 1) * cw + m;
+  const double a = (double)h.a, UL = (double)h.UL, cw = 1.0 / (double)h.inv_cw, m = kCellMargin * cw;
+  const double lo_x = axis_inv(a, ix * cw - UL - m), hi_x = axis_inv(a, (ix + 1) * cw - UL + m);
+  const double lo_y = axis_inv(a, iy * cw - UL - m), hi_y = axis_inv(a, (iy + 1) * cw - UL + m);
+  x0 = lo_x - 1e-12 * fabs(lo_x);
+  x1 = hi_x + 1e-12 * fabs(hi_x);
+  y0 = lo_y - 1e-12 * fabs(lo_y);
+  y1 = hi_y + 1e-12 * fabs(hi_y);
 }
 
 __device__ __forceinline__ double dmax2(double cx, double cy, double x0, double x1, double y0, double y1) {
