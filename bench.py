@@ -512,7 +512,12 @@ def run_ours(args):
     if brute_roof is not None:
         rooflines["encode_brute_force"] = brute_roof
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers. Every step
+    # copies its inputs (W, act RMS) from pinned host memory and reads back its
+    # results (decoded bf16 matrix, packed stream, r, s, sigma). Steps are
+    # pipelined over two buffer slots and three streams (host-to-device copy,
+    # compute, device-to-host copy), so step i+1's upload and step i-1's
+    # read-back overlap step i's kernels, as a stream of matrices would run.
     e2e = None
     if not args.no_e2e:
         Wh = Wt.pin_memory()
@@ -522,32 +527,64 @@ def run_ours(args):
         rh = torch.empty(M, dtype=torch.float32).pin_memory()
         sh = torch.empty(K, dtype=torch.float32).pin_memory()
         sgh = torch.empty(K // 2, dtype=torch.float32).pin_memory()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        slots = []
+        for _ in range(2):
+            slots.append(dict(
+                W=torch.empty_like(Wd), act=torch.empty_like(actd), ws=torch.empty_like(ws),
+                sigma=torch.empty_like(sigma), packed=torch.empty_like(packed), r=torch.empty_like(rnorm),
+                s=torch.empty_like(cscale), out=torch.empty_like(out),
+                h2d=torch.cuda.Event(), comp=torch.cuda.Event(), d2h=torch.cuda.Event()))
+        s_h2d, s_comp, s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
 
-        def e2e_step():
-            Wd.copy_(Wh, non_blocking=True)
-            actd.copy_(acth, non_blocking=True)
-            one()
-            outh.copy_(out, non_blocking=True)
-            pkh.copy_(packed, non_blocking=True)
-            rh.copy_(rnorm, non_blocking=True)
-            sh.copy_(cscale, non_blocking=True)
-            sgh.copy_(sigma, non_blocking=True)
+        def e2e_step(i):
+            sl = slots[i % 2]
+            with torch.cuda.stream(s_h2d):
+                s_h2d.wait_event(sl["comp"])            # step i-2 has finished reading this slot's inputs
+                sl["W"].copy_(Wh, non_blocking=True)
+                sl["act"].copy_(acth, non_blocking=True)
+                sl["h2d"].record(s_h2d)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(sl["h2d"])
+                s_comp.wait_event(sl["d2h"])            # step i-2's results have been read back
+                sg = q.calibrate_sigma(sl["W"], sl["act"], spec.alpha, spec.block, spec.seed, status=status,
+                                       workspace=sl["ws"], out=sl["sigma"], stream=s_comp)
+                enc = q.encode(sl["W"], sl["act"], spec.alpha, spec.block, spec.seed, sg, Cd, spec.bits,
+                               status=status, out=(sl["packed"], sl["r"], sl["s"]), search_table=table,
+                               stream=s_comp)
+                q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=sl["out"], stream=s_comp)
+                sl["comp"].record(s_comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(sl["comp"])
+                outh.copy_(sl["out"], non_blocking=True)
+                pkh.copy_(sl["packed"], non_blocking=True)
+                rh.copy_(sl["r"], non_blocking=True)
+                sh.copy_(sl["s"], non_blocking=True)
+                sgh.copy_(sl["sigma"], non_blocking=True)
+                sl["d2h"].record(s_d2h)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        for i in range(max(2, args.warmup)):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        for st in (s_h2d, s_comp, s_d2h):
+            st.wait_event(e0)
+        for i in range(args.steps):
+            e2e_step(i)
+        stream.wait_stream(s_d2h)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+        if status.item() != 0:
+            raise SystemExit(f"device status {status.item()} in the end-to-end steps")
+        if not torch.equal(pkh, packed.cpu()):
+            raise SystemExit("end-to-end packed stream differs from the device-resident run")
         e2e = {"value": aggregate_throughput(weights * args.steps, e2e_s, world) / 1e9, "unit": "Gweights/s",
                "h2d_bytes_per_step": Wh.numel() * 2 + acth.numel() * 4,
-               "d2h_bytes_per_step": outh.numel() * 2 + pkh.numel() * 4 + 4 * M + 4 * K + 2 * K}
+               "d2h_bytes_per_step": outh.numel() * 2 + pkh.numel() * 4 + 4 * M + 4 * K + 2 * K,
+               "pipelining": "2 buffer slots; H2D, compute and D2H on three streams"}
 
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None

@@ -96,6 +96,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t t0 = (int64_t)blockIdx.x * T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
   const double inv_sqrt_b = 1.0 / sqrt((double)(1 << ra.log2b));
   const int B = a.bits;
+  // floor(n / B) = (n * divB) >> 32 exactly for 0 <= n < 2^14 and 1 <= B <= 16
+  // (checked exhaustively); the packing needs n < 256 * 16 + 32
+  const uint64_t divB = (0x100000000ull / (uint64_t)B) + 1ull;
 
   // the next unit's weights and row norm, loaded while the current one is searched
   auto prefetch = [&](int64_t t, WRegs<WT> &w, float &rn) -> bool {
@@ -161,23 +164,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
 
-    // candidate ranges of the 8 pairs (cell lists, or the identity list)
+    // candidate ranges of the 8 pairs (cell lists, or the identity list),
+    // without branches: an off-grid pair reads cell 0 and discards it
     int beg[8], end[8];
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
-      beg[p] = 0;
-      end[p] = N;
-      if (use) {
-        const float u0 = __fdividef(x0[p], __fadd_rn(a_ax, fabsf(x0[p])));
-        const float u1 = __fdividef(x1[p], __fadd_rn(a_ax, fabsf(x1[p])));
-        const float fx = __fmul_rn(__fadd_rn(u0, UL), inv_cw);
-        const float fy = __fmul_rn(__fadd_rn(u1, UL), inv_cw);
-        if (fx >= 0.0f && fx < Gf && fy >= 0.0f && fy < Gf) {
-          const int cell = (int)fy * G + (int)fx;
-          beg[p] = toff[cell];
-          end[p] = toff[cell + 1];
-        }
-      }
+      const float u0 = __fdividef(x0[p], __fadd_rn(a_ax, fabsf(x0[p])));
+      const float u1 = __fdividef(x1[p], __fadd_rn(a_ax, fabsf(x1[p])));
+      const float fx = __fmul_rn(__fadd_rn(u0, UL), inv_cw);
+      const float fy = __fmul_rn(__fadd_rn(u1, UL), inv_cw);
+      const bool in = use && fx >= 0.0f && fx < Gf && fy >= 0.0f && fy < Gf;
+      const int cell = in ? (int)fy * G + (int)fx : 0;
+      const int b0 = toff[cell], e0 = toff[cell + 1];
+      beg[p] = in ? b0 : 0;
+      end[p] = in ? e0 : N;
     }
     int idx[8];
 #pragma unroll
@@ -207,8 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *dst = a.packed + row * a.wpr + chunk * (int64_t)(8 * B);
     for (int w = lane; w < nw; w += 32) {
       const int bit0 = w * 32;
-      const int k0 = bit0 / B;
-      const int k1 = min((bit0 + 31) / B, np - 1);
+      const int k0 = (int)(((uint64_t)bit0 * divB) >> 32);               // bit0 / B
+      const int k1 = min((int)(((uint64_t)(bit0 + 31) * divB) >> 32), np - 1);
       uint32_t word = 0;
       for (int k = k0; k <= k1; ++k) {
         const int off = k * B - bit0;
