@@ -3,7 +3,7 @@
 // Same arithmetic as qamw_decode.cu ("QAM-W: Joint 2D Codebook Quantization
 // for LLM Weights ...", Methodology (6) Decoding), different data movement:
 //   * packed words reach shared memory through one 2D TMA tensor load per
-//     task (a box of ROWS rows x SEGS*128 columns worth of words), double
+//     task (a box of ROWS rows x SEGS*64 columns worth of words), double
 //     buffered and tracked by an mbarrier per stage;
 //   * bf16 results are written into a 128-byte-swizzled staging tile and leave
 //     through 2D TMA tensor stores (one per 64 columns), which clip rows and
@@ -13,11 +13,15 @@
 // loads touched one sector per lane; the coalescing copy-out doubled the
 // shared-memory traffic of the staging).
 //
-// Task geometry: a warp decodes ROWS rows x SEGS segments of 128 columns with
-// lane = row + ROWS * segment. SEGS = b/128 for b > 128; otherwise 1, or 2
-// when one segment's words (8*bits bytes) are not a multiple of 16 bytes
-// (a TMA box row must be). Each lane owns one segment of one row, as in the
-// plain kernel.
+// Task geometry: a warp decodes ROWS rows x SEGS segments of 64 columns with
+// lane = row + ROWS * segment; each lane owns one segment of one row: 32
+// indices, i.e. exactly `bits` packed words starting on a word boundary, and
+// 64 fp32 values (about 100 registers, 16 warps per SM). SEGS is the larger
+// of b/64 (the lanes of one block) and the segments whose words make a
+// multiple of 16 bytes (a TMA box row must): 1 for bits % 4 == 0, 2 for even
+// bits, 4 for odd bits. Block bits 1..5 are butterflies inside the lane, bits
+// >= 6 across lanes (lane xor ROWS << (t - 6)) as fma(+-1, own, partner's),
+// which rounds exactly like the add or subtract.
 //
 // Every mbarrier wait is bounded; a wait that runs out sets
 // QAMW_STATUS_TIMEOUT and the kernel stops issuing work.
@@ -34,8 +38,8 @@
 namespace qamw {
 namespace {
 
-constexpr int kSeg = 128;
-constexpr int kMaxWarps = 12;
+constexpr int kSeg = 64;
+constexpr int kMaxWarps = 16;
 constexpr uint32_t kWaitLimit = 1u << 22;   // try_wait attempts before giving up
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -113,25 +117,30 @@ __device__ __forceinline__ void inlane_stages(float (&v)[kSeg]) {
   if constexpr (LB > 3) bfly_stage<3>(v);
   if constexpr (LB > 4) bfly_stage<4>(v);
   if constexpr (LB > 5) bfly_stage<5>(v);
-  if constexpr (LB > 6) bfly_stage<6>(v);
 }
 
+// Block bit TB >= 6 across lanes: the partner holds the same columns of the
+// other half; the lower lane keeps own + partner's, the upper partner's - own.
 template <int TB, int ROWS>
 __device__ __forceinline__ void xlane_stage(float (&v)[kSeg], int lane) {
-  constexpr int h = ROWS << (TB - 7);
-  const bool upper = (lane & h) != 0;
+  constexpr int h = ROWS << (TB - 6);
+  const float sg = (lane & h) ? -1.0f : 1.0f;
+  const float2 S = make_float2(sg, sg);
 #pragma unroll
-  for (int i = 0; i < kSeg; ++i) {
-    const float p = __shfl_xor_sync(0xffffffffu, v[i], h);
-    v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+  for (int i = 0; i < kSeg; i += 2) {
+    const float2 V = make_float2(v[i], v[i + 1]);
+    const float2 P = make_float2(__shfl_xor_sync(0xffffffffu, v[i], h), __shfl_xor_sync(0xffffffffu, v[i + 1], h));
+    const float2 o = fma2(S, V, P);
+    v[i] = o.x;
+    v[i + 1] = o.y;
   }
 }
 
 template <int LB, int ROWS>
 __device__ __forceinline__ void xlane_stages(float (&v)[kSeg], int lane) {
+  if constexpr (LB > 6) xlane_stage<6, ROWS>(v, lane);
   if constexpr (LB > 7) xlane_stage<7, ROWS>(v, lane);
   if constexpr (LB > 8) xlane_stage<8, ROWS>(v, lane);
-  if constexpr (LB > 9) xlane_stage<9, ROWS>(v, lane);
 }
 
 #ifndef QAMW_DEC_STAGES
@@ -141,19 +150,21 @@ constexpr int kStages = QAMW_DEC_STAGES;   // input pipeline depth; 1 measured f
 
 template <int BITS, int LB>
 struct TmaGeom {
-  static constexpr int kSegs = (LB > 7) ? (1 << (LB - 7)) : ((BITS & 1) ? 2 : 1);
+  static constexpr int kSegsBlock = (LB > 6) ? (1 << (LB - 6)) : 1;
+  static constexpr int kSegsAlign = (BITS % 4 == 0) ? 1 : ((BITS % 2 == 0) ? 2 : 4);
+  static constexpr int kSegs = (kSegsBlock > kSegsAlign) ? kSegsBlock : kSegsAlign;
   static constexpr int kRows = 32 / kSegs;
   static constexpr int kLog2Rows = (kRows == 32) ? 5 : (kRows == 16) ? 4 : (kRows == 8) ? 3 : 2;
-  static constexpr int kBoxWords = kSegs * 2 * BITS;          // words per row of the input box
+  static constexpr int kBoxWords = kSegs * BITS;              // words per row of the input box
   static constexpr int kInBytes = kRows * kBoxWords * 4;      // one input stage
-  static constexpr int kOutBoxes = kSegs * 2;                 // 64-column output boxes per task
+  static constexpr int kOutBoxes = kSegs;                     // 64-column output boxes per task
   static constexpr int kOutBoxBytes = kRows * 128;            // one swizzled output box
   // per-warp layout (byte offsets); the staging tile first (1024-byte aligned)
   static constexpr int kOffStage = 0;
   static constexpr int kOffIn = kOffStage + kOutBoxes * kOutBoxBytes;
   static constexpr int kStageBytes = kInBytes + ((kRows * 4 + 127) & ~127);  // words + row norms
-  static constexpr int kOffCf = kOffIn + kStages * kStageBytes;        // kSegs x (128 + 4) floats
-  static constexpr int kOffSg = kOffCf + kSegs * (kSeg + 4) * 4;       // kSegs x (64 + 2) float2
+  static constexpr int kOffCf = kOffIn + kStages * kStageBytes;        // kSegs x (64 + 4) floats
+  static constexpr int kOffSg = kOffCf + kSegs * (kSeg + 4) * 4;       // kSegs x (32 + 2) float2
   static constexpr int kOffBar = kOffSg + kSegs * (kSeg / 2 + 2) * 8;  // kStages mbarriers
   static constexpr int kWarpBytes = (kOffBar + 8 * kStages + 1023) & ~1023;
 };
@@ -169,7 +180,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     decode_tma_kernel(TmaArgs ta, const __grid_constant__ CUtensorMap in_map,
                       const __grid_constant__ CUtensorMap rn_map, const __grid_constant__ CUtensorMap out_map) {
   using G = TmaGeom<BITS, LB>;
-  constexpr int SEGS = G::kSegs, ROWS = G::kRows, NW = 2 * BITS;
+  constexpr int SEGS = G::kSegs, ROWS = G::kRows, NW = BITS;
   const DecodeArgs &a = ta.a;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -258,12 +269,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
           if (mask_is_negative(a.seed, col)) v = -v;
           f = (float)v;
         }
-        cf[(j >> 7) * (kSeg + 4) + (j & 127)] = f;
+        cf[(j >> 6) * (kSeg + 4) + (j & 63)] = f;
       }
       for (int p = lane; p < SEGS * kSeg / 2; p += 32) {
         const int64_t k = (colbase >> 1) + p;
         const float sk = (k < P) ? a.sigma[k] : 0.0f;
-        sg[(p >> 6) * (kSeg / 2 + 2) + (p & 63)] = make_float2(sk, sk);
+        sg[(p >> 5) * (kSeg / 2 + 2) + (p & 31)] = make_float2(sk, sk);
       }
       __syncwarp();
       cur = segcol;
@@ -283,11 +294,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
     uint32_t w[NW + 1];
     const uint32_t *wsrc = inbuf + rr * G::kBoxWords + sgi * NW;
 #pragma unroll
-    for (int i = 0; i < NW / 2; ++i) {
-      const uint2 u = *reinterpret_cast<const uint2 *>(wsrc + 2 * i);
-      w[2 * i] = u.x;
-      w[2 * i + 1] = u.y;
-    }
+    for (int i = 0; i < NW; ++i) w[i] = wsrc[i];
     w[NW] = 0u;
     __syncwarp();
     if (lane == 0 && t + kStages < t1) {
@@ -346,10 +353,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       pk.y = *reinterpret_cast<uint32_t *>(&b1);
       pk.z = *reinterpret_cast<uint32_t *>(&b2);
       pk.w = *reinterpret_cast<uint32_t *>(&b3);
-      // column c of this lane's segment -> output box 2*sgi + c/64, 16-byte chunk (c%64)/8,
+      // column c of this lane's segment -> output box sgi, 16-byte chunk c/8,
       // stored at chunk ^ (row % 8) (the 128-byte swizzle of the TMA box)
-      const int box = 2 * sgi + (c >> 6);
-      const int chunk = ((c & 63) >> 3) ^ (rr & 7);
+      const int box = sgi;
+      const int chunk = (c >> 3) ^ (rr & 7);
       *reinterpret_cast<uint4 *>(stage + box * G::kOutBoxBytes + rr * 128 + chunk * 16) = pk;
     }
     fence_proxy_async();
@@ -473,8 +480,10 @@ bool decode_tma_applicable(const DecodeArgs &a) {
   if (a.M > (int64_t(1) << 30) || a.wpr > (int64_t(1) << 30)) return false;
   if (reinterpret_cast<uintptr_t>(a.row_norm) % 16) return false;
   // task indices are 32-bit
-  const int64_t segs = (a.log2b > 7) ? (int64_t(1) << (a.log2b - 7)) : ((a.bits & 1) ? 2 : 1);
-  if (((a.K + segs * 128 - 1) / (segs * 128)) * ((a.M + 31) / (32 / segs)) > (int64_t(1) << 30)) return false;
+  const int64_t sb = (a.log2b > 6) ? (int64_t(1) << (a.log2b - 6)) : 1;
+  const int64_t sa = (a.bits % 4 == 0) ? 1 : ((a.bits % 2 == 0) ? 2 : 4);
+  const int64_t segs = sb > sa ? sb : sa;
+  if (((a.K + segs * 64 - 1) / (segs * 64)) * ((a.M + 31) / (32 / segs)) > (int64_t(1) << 30)) return false;
   return tensor_map_encoder() != nullptr;
 }
 
