@@ -50,7 +50,11 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    p.add_argument("--workload", default="llama7b_attn", choices=("llama7b_attn", "tiny", "decode_13b"))
+    p.add_argument("--workload", default="llama7b_attn",
+                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4"),
+                   help="llama7b_attn: 4096x4096 bf16 at 2048 centroids (5.5 bits/weight; the default); "
+                        "rate35 / rate4: the same matrix at 128 / 256 centroids (3.5 / 4 bits/weight); "
+                        "decode_13b: decode-only sweep over the 13B shapes; tiny: 256x512 fp32")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
@@ -499,6 +503,9 @@ def run_ours(args):
                     "unit": "Gop/s", "frac": ops / (enc_ms * 1e-3) / fp32_peak, "traffic": None,
                     "kernel": "encode_pruned_kernel (exact pruned search; events span the qamw_encode call)",
                     "evaluations_per_pair": evals / P, "peak_source": fp32_src,
+                    "brute_force_equivalent_frac": 4.0 * P * spec.N / (enc_ms * 1e-3) / fp32_peak,
+                    "brute_force_equivalent_note": "the FP32 work a brute-force search would do in the same time; "
+                                                   "above 1 because the pruned search skips it",
                     "hbm_gbs": (M * K * 2 + M * wpr * 4) / (enc_ms * 1e-3) / 1e9}
     else:
         enc_roof = brute_roof

@@ -27,7 +27,7 @@ import numpy as np
 __all__ = [
     "MatrixSpec", "Workload", "make_matrix", "make_act_rms", "make_indices",
     "make_row_norms", "make_sigma", "to_bf16", "tiny", "llama7b_attn", "mlp_runs",
-    "stack_1p1b", "decode_sweep_13b", "WORKLOADS",
+    "stack_1p1b", "decode_sweep_13b", "rate_variant", "WORKLOADS",
 ]
 
 
@@ -173,8 +173,18 @@ def decode_sweep_13b() -> Workload:
         _spec("13b.down", 5120, 13824, seed=5002)], ops=("decode",))
 
 
+def rate_variant(bits: int) -> Workload:
+    """The lower-rate codecs on the 4096 x 4096 projection (same matrix recipe):
+    3.5 bits/weight (128 centroids, 7 bits per pair) and 4 bits/weight (256
+    centroids, 8 bits per pair)."""
+    N = 1 << bits
+    return Workload(f"llama7b_attn_4096x4096_bf16_b128_N{N}", [
+        _spec("attn", 4096, 4096, out=0.005, out_scale=20.0, N=N, bits=bits, seed=2000)])
+
+
 WORKLOADS = {"tiny": tiny, "llama7b_attn": llama7b_attn, "mlp": mlp_runs,
-             "stack_1p1b": stack_1p1b, "decode_13b": decode_sweep_13b}
+             "stack_1p1b": stack_1p1b, "decode_13b": decode_sweep_13b,
+             "rate35": lambda: rate_variant(7), "rate4": lambda: rate_variant(8)}
 
 
 def act_for(spec: MatrixSpec) -> np.ndarray:

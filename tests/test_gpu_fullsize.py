@@ -66,6 +66,16 @@ def test_mlp_projection_runs(which):
     _check_encode(spec, n_rows=6)
 
 
+@pytest.mark.parametrize("bits", [7, 8])
+def test_rate_variants_on_the_projection(bits):
+    """QAM-W at 3.5 and 4 bits per weight (128 and 256 centroids) on the 4096x4096
+    projection: encode through the pruned search, and the bf16 decode path of
+    7- and 8-bit words."""
+    spec = synth.rate_variant(bits).specs[0]
+    _check_encode(spec, n_rows=10)
+    _check_decode_random(spec.M, spec.K, spec.block, spec.N, spec.bits, spec.seed, rows=_sample_rows(spec.M, 8, 1))
+
+
 def test_stack_layer0():
     for spec in synth.stack_1p1b(1).specs:
         _check_encode(spec, n_rows=4)
