@@ -51,10 +51,11 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="llama7b_attn",
-                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4"),
+                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4", "lloyd"),
                    help="llama7b_attn: 4096x4096 bf16 at 2048 centroids (5.5 bits/weight; the default); "
                         "rate35 / rate4: the same matrix at 128 / 256 centroids (3.5 / 4 bits/weight); "
-                        "decode_13b: decode-only sweep over the 13B shapes; tiny: 256x512 fp32")
+                        "decode_13b: decode-only sweep over the 13B shapes; tiny: 256x512 fp32; "
+                        "lloyd: codebook training, one Lloyd iteration of 2048 centroids on 2^21 samples per step")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
@@ -366,9 +367,97 @@ def run_decode_sweep(args):
     return 0
 
 
+LLOYD_N, LLOYD_T, LLOYD_SEED = 2048, 1 << 21, 12345 + 2048
+FP64_LANES_PER_SM = 64
+
+
+def run_lloyd(args):
+    """Steps of codebook training: one Lloyd iteration (qamw_lloyd_update then
+    qamw_lloyd_assign) of 2048 centroids on 2^21 unit-Gaussian samples -- the
+    size the shipped 2048-centroid codebook was trained at. Each iteration is
+    timed with CUDA events; the start is the first 2048 samples."""
+    import torch
+    import synth
+    import vector_codebook_codec_b200 as q
+    from vector_codebook_codec_b200 import build as qbuild
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qbuild.build()
+    x = synth.gaussian_points(LLOYD_T, LLOYD_SEED)
+    pts = torch.from_numpy(x).to(dev)
+    C = pts[:LLOYD_N].clone()
+    lib = q.load_library()
+    idx = torch.full((LLOYD_T,), -1, dtype=torch.int32, device=dev)
+    ws = torch.empty(int(lib.qamw_lloyd_workspace_bytes(LLOYD_T, LLOYD_N)), dtype=torch.uint8, device=dev)
+    changed = torch.zeros(1, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    q.lloyd_assign(pts, C, idx=idx)
+
+    def one():
+        q._check("qamw_lloyd_update", lib.qamw_lloyd_update(q._ptr(pts), LLOYD_T, q._ptr(idx), LLOYD_N, q._ptr(C),
+                                                            q._ptr(ws), ws.numel(), q._stream_ptr(stream)))
+        q.lloyd_assign(pts, C, idx=idx, changed=changed)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    total_s = sum(ms) / 1e3
+    value = args.steps / total_s
+    peaks, peak_kind = measured_peaks()
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    fp64_peak = sms * FP64_LANES_PER_SM * sm_max * 1e6
+    ops = 5.0 * LLOYD_T * LLOYD_N          # 2 fp64 subs, 2 muls, 1 add per (sample, centroid)
+    mean_s = total_s / args.steps
+    roof = {"bound": "alu", "achieved": ops / mean_s / 1e9, "peak": fp64_peak / 1e9, "unit": "Gop/s",
+            "frac": ops / mean_s / fp64_peak, "traffic": None,
+            "kernel": "lloyd_assign_kernel + lloyd_partial_kernel + lloyd_reduce_kernel (events span one iteration)",
+            "peak_source": f"{sms} SMs x {FP64_LANES_PER_SM} FP64 lanes x {sm_max:.0f} MHz ({peak_kind} max clock)"}
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        from oracle import lloyd as olloyd
+        Ts = 1 << 18
+        xs, Cs = x[:Ts], x[:LLOYD_N].copy()
+        i0 = olloyd.assign(xs, Cs)
+        t0 = time.perf_counter()
+        reps = 3
+        for _ in range(reps):
+            Cs = olloyd.centroid_update(xs, i0, Cs)
+            i0 = olloyd.assign(xs, Cs)
+        dt = (time.perf_counter() - t0) / reps
+        cpu = {"value": (Ts / LLOYD_T) / dt, "unit": "iterations/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"{Ts} of {LLOYD_T} samples per iteration (cKDTree assignment on all cores + bincount "
+                         f"means), scaled to the full sample count"}
+    if rank == 0:
+        line = {"metric": "QAM-W codebook training: Lloyd iterations per second", "value": value,
+                "unit": "iterations/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * mean_s, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic (seeded unit circular Gaussian samples)",
+                "config": {"workload": "lloyd_N2048_T2097152", "N": LLOYD_N, "T": LLOYD_T, "seed": LLOYD_SEED,
+                           "l2": "samples (32 MB) stay in L2 between iterations; the work is ALU-bound"},
+                "roofline": roof, "cpu_baseline": cpu, "gpu_launches": 3 * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args):
     if args.workload == "decode_13b":
         return run_decode_sweep(args)
+    if args.workload == "lloyd":
+        return run_lloyd(args)
     import torch
     import torch.distributed as dist
 

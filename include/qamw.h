@@ -220,6 +220,42 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
 int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t block,
                      uint64_t sign_seed, int32_t inverse, qamw_stream_t stream);
 
+/*
+ * Lloyd training of the 2D codebook -- Methodology (4) Joint 2D Quantization
+ * and "Significance and Claims" (the codebook is a 2D Lloyd-Max quantizer
+ * trained once on samples of the unit circular Gaussian). One iteration:
+ * assign every sample to its nearest centroid (Euclidean, lowest index on
+ * ties), then move every centroid to the mean of its samples (a centroid
+ * with no sample keeps its place). Everything is fp64.
+ *   points    : device float64 [T][2], 16-byte aligned (the samples; drawn by
+ *               the caller)
+ *   centroids : device float64 [N][2], 16-byte aligned, 1 <= N <= QAMW_MAX_CENTROIDS
+ *   idx       : device int32 [T]
+ *   workspace : device, 256-byte aligned, >= qamw_lloyd_workspace_bytes(T, N)
+ * Sums are formed in a fixed order, so results do not depend on the device.
+ *
+ * qamw_lloyd_assign writes the nearest index of every sample into idx_inout
+ * and, if `changed` (device uint64) is not NULL, adds the number of samples
+ * whose index differs from what idx_inout held before.
+ * qamw_lloyd_update moves the centroids (in place) to the means of their
+ * samples under idx.
+ * qamw_lloyd_train runs idx = assign(C); then, up to max_iter times,
+ * C = update(idx), idx' = assign(C), stopping when no index changed. It writes
+ * the trained centroids in place, the final assignment, and (host pointers,
+ * nullable) the iteration count and whether it converged. It synchronizes
+ * `stream` once per iteration.
+ * Errors: QAMW_ENULL, QAMW_EINVAL (T < 1, N out of range, alignment,
+ * max_iter < 0), QAMW_EWORKSPACE, QAMW_ECUDA.
+ */
+size_t qamw_lloyd_workspace_bytes(int64_t T, int32_t N);
+int qamw_lloyd_assign(const double *points, int64_t T, const double *centroids, int32_t N, int32_t *idx_inout,
+                      unsigned long long *changed, qamw_stream_t stream);
+int qamw_lloyd_update(const double *points, int64_t T, const int32_t *idx, int32_t N, double *centroids_inout,
+                      void *workspace, size_t workspace_bytes, qamw_stream_t stream);
+int qamw_lloyd_train(const double *points, int64_t T, double *centroids, int32_t N, int32_t max_iter,
+                     int32_t *idx_out, void *workspace, size_t workspace_bytes, int32_t *iterations_out,
+                     int32_t *converged_out, qamw_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

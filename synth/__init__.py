@@ -27,7 +27,7 @@ import numpy as np
 __all__ = [
     "MatrixSpec", "Workload", "make_matrix", "make_act_rms", "make_indices",
     "make_row_norms", "make_sigma", "to_bf16", "tiny", "llama7b_attn", "mlp_runs",
-    "stack_1p1b", "decode_sweep_13b", "rate_variant", "WORKLOADS",
+    "stack_1p1b", "decode_sweep_13b", "rate_variant", "gaussian_points", "WORKLOADS",
 ]
 
 
@@ -99,6 +99,12 @@ def make_indices(M: int, P: int, N: int, seed: int) -> np.ndarray:
 def make_row_norms(M: int, seed: int) -> np.ndarray:
     """Positive float32 row norms ~ 0.02*sqrt(K)-sized, for decode-only inputs."""
     return (np.exp(_rng(seed + 1).standard_normal(M) * 0.25) * 1.0).astype(np.float32)
+
+
+def gaussian_points(T: int, seed: int) -> np.ndarray:
+    """T draws of the unit circular Gaussian N(0, I_2), float64 [T, 2] (PCG64
+    standard normals, row-major): the training samples of a 2D codebook."""
+    return _rng(seed).standard_normal((T, 2))
 
 
 def make_sigma(P: int, seed: int) -> np.ndarray:

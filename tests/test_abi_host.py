@@ -137,3 +137,24 @@ def test_error_message_cleared_on_next_rejection(lib):
     assert _enc(lib, K=255, ldw=255) == QAMW_EINVAL
     assert lib.qamw_last_error() != first and b"K" in lib.qamw_last_error()
     assert QAMW_OK == 0
+
+
+def test_lloyd_entry_points_reject_on_host(lib):
+    ws = 1 << 30
+    assert lib.qamw_lloyd_workspace_bytes(0, 16) == 0
+    assert lib.qamw_lloyd_workspace_bytes(1000, 16) >= 3 * 8 * 16 + 8
+    assert lib.qamw_lloyd_assign(None, 10, FAKE, 4, FAKE, None, None) == QAMW_ENULL
+    assert lib.qamw_lloyd_assign(FAKE, 10, FAKE, 4, None, None, None) == QAMW_ENULL
+    assert lib.qamw_lloyd_assign(FAKE, 0, FAKE, 4, FAKE, None, None) == QAMW_EINVAL
+    assert lib.qamw_lloyd_assign(FAKE, 10, FAKE, 0, FAKE, None, None) == QAMW_EINVAL
+    assert lib.qamw_lloyd_assign(FAKE, 10, FAKE, 8193, FAKE, None, None) == QAMW_EINVAL
+    assert lib.qamw_lloyd_assign(ctypes.c_void_p(0x10008), 10, FAKE, 4, FAKE, None, None) == QAMW_EINVAL
+    assert lib.qamw_lloyd_update(FAKE, 10, FAKE, 4, FAKE, None, ws, None) == QAMW_EWORKSPACE
+    assert lib.qamw_lloyd_update(FAKE, 10, FAKE, 4, FAKE, FAKE, 8, None) == QAMW_EWORKSPACE
+    assert lib.qamw_lloyd_update(FAKE, 10, None, 4, FAKE, FAKE, ws, None) == QAMW_ENULL
+    assert lib.qamw_lloyd_update(FAKE, 10, FAKE, 4, FAKE, ctypes.c_void_p(0x10010), ws, None) == QAMW_EINVAL
+    it, conv = ctypes.c_int32(-5), ctypes.c_int32(-5)
+    assert lib.qamw_lloyd_train(FAKE, 10, FAKE, 4, -1, FAKE, FAKE, ws, ctypes.byref(it), ctypes.byref(conv),
+                                None) == QAMW_EINVAL
+    assert lib.qamw_lloyd_train(FAKE, 10, FAKE, 4, 5, None, FAKE, ws, None, None, None) == QAMW_ENULL
+    assert it.value == -5 and conv.value == -5   # untouched on a rejected call

@@ -54,6 +54,10 @@ _SIGNATURES = {
     "qamw_build_search_table": (ctypes.c_int, [_c_p, _c_i32, _c_p, _c_sz, _c_p]),
     "qamw_calibrate_sigma_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
                                                     _c_i32, _c_u64, _c_p, _c_p, _c_p]),
+    "qamw_lloyd_workspace_bytes": (_c_sz, [_c_i64, _c_i32]),
+    "qamw_lloyd_assign": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_p]),
+    "qamw_lloyd_update": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_sz, _c_p]),
+    "qamw_lloyd_train": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_sz, _c_p, _c_p, _c_p]),
 }
 
 _lib = None
@@ -109,6 +113,10 @@ qamw_calibrate_sigma = _raw("qamw_calibrate_sigma")
 qamw_encode = _raw("qamw_encode")
 qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
+qamw_lloyd_workspace_bytes = _raw("qamw_lloyd_workspace_bytes")
+qamw_lloyd_assign = _raw("qamw_lloyd_assign")
+qamw_lloyd_update = _raw("qamw_lloyd_update")
+qamw_lloyd_train = _raw("qamw_lloyd_train")
 qamw_calibrate_sigma_noalloc = _raw("qamw_calibrate_sigma_noalloc")
 qamw_search_table_bytes = _raw("qamw_search_table_bytes")
 qamw_build_search_table = _raw("qamw_build_search_table")
@@ -286,3 +294,63 @@ def rotate_rows(U, block: int, seed: int, inverse: bool = False, stream=None):
     _check("qamw_rotate_rows", load_library().qamw_rotate_rows(
         _ptr(U), _ptr(Y), M, K, block, seed & (2**64 - 1), 1 if inverse else 0, _stream_ptr(stream)))
     return Y
+
+
+# ---------------------------------------------------------------------------
+# Lloyd training of the 2D codebook (qamw_lloyd_*)
+# ---------------------------------------------------------------------------
+
+def _lloyd_inputs(points, centroids):
+    torch = _torch()
+    _need_cuda("points", points, torch.float64, 2)
+    _need_cuda("centroids", centroids, torch.float64, 2)
+    if points.shape[1] != 2 or centroids.shape[1] != 2:
+        raise ValueError("points and centroids must be [.][2]")
+    return points.contiguous(), centroids.contiguous()
+
+
+def _lloyd_workspace(lib, T, N, device):
+    torch = _torch()
+    need = int(lib.qamw_lloyd_workspace_bytes(T, N))
+    return torch.empty(need, dtype=torch.uint8, device=device), need
+
+
+def lloyd_assign(points, centroids, idx=None, changed=None, stream=None):
+    """Nearest centroid (fp64, lowest index on ties) of every point; int32 [T]."""
+    torch = _torch()
+    points, centroids = _lloyd_inputs(points, centroids)
+    T, N = points.shape[0], centroids.shape[0]
+    if idx is None:
+        idx = torch.full((T,), -1, dtype=torch.int32, device=points.device)
+    _check("qamw_lloyd_assign", load_library().qamw_lloyd_assign(
+        _ptr(points), T, _ptr(centroids), N, _ptr(idx), _ptr(changed), _stream_ptr(stream)))
+    return idx
+
+
+def lloyd_update(points, idx, centroids, stream=None):
+    """Moves the centroids (fp64 [N][2] CUDA tensor, in place) to the means of their points."""
+    points, c = _lloyd_inputs(points, centroids)
+    if c.data_ptr() != centroids.data_ptr():
+        raise ValueError("centroids must be contiguous (updated in place)")
+    lib = load_library()
+    ws, need = _lloyd_workspace(lib, points.shape[0], c.shape[0], points.device)
+    _check("qamw_lloyd_update", lib.qamw_lloyd_update(
+        _ptr(points), points.shape[0], _ptr(idx), c.shape[0], _ptr(c), _ptr(ws), need, _stream_ptr(stream)))
+    return centroids
+
+
+def lloyd_train(points, init, max_iter: int = 500, stream=None):
+    """Lloyd iterations from ``init`` (fp64 [N][2]) on ``points`` (fp64 [T][2]).
+    Returns (centroids, idx, iterations, converged); see qamw_lloyd_train."""
+    torch = _torch()
+    points, init = _lloyd_inputs(points, init)
+    C = init.clone()
+    T, N = points.shape[0], C.shape[0]
+    idx = torch.empty(T, dtype=torch.int32, device=points.device)
+    lib = load_library()
+    ws, need = _lloyd_workspace(lib, T, N, points.device)
+    it, conv = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("qamw_lloyd_train", lib.qamw_lloyd_train(
+        _ptr(points), T, _ptr(C), N, int(max_iter), _ptr(idx), _ptr(ws), need, ctypes.byref(it),
+        ctypes.byref(conv), _stream_ptr(stream)))
+    return C, idx, int(it.value), bool(conv.value)

@@ -266,4 +266,87 @@ int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t b
   return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
 }
 
+size_t qamw_lloyd_workspace_bytes(int64_t T, int32_t N) {
+  if (T < 1 || N < 1 || N > QAMW_MAX_CENTROIDS) return 0;
+  return qamw::lloyd_workspace_bytes(T, N);
+}
+
+static int check_lloyd(const void *points, int64_t T, const void *centroids, int32_t N, const char *fn) {
+  if (!points || !centroids) return fail(QAMW_ENULL, "%s: points and centroids must be non-NULL", fn);
+  if (T < 1) return fail(QAMW_EINVAL, "%s: T (%lld) must be >= 1", fn, (long long)T);
+  if (N < 1 || N > QAMW_MAX_CENTROIDS)
+    return fail(QAMW_EINVAL, "%s: N (%d) must be in [1, %d]", fn, N, QAMW_MAX_CENTROIDS);
+  if (reinterpret_cast<uintptr_t>(points) % 16 || reinterpret_cast<uintptr_t>(centroids) % 16)
+    return fail(QAMW_EINVAL, "%s: points and centroids must be 16-byte aligned", fn);
+  return QAMW_OK;
+}
+
+int qamw_lloyd_assign(const double *points, int64_t T, const double *centroids, int32_t N, int32_t *idx_inout,
+                      unsigned long long *changed, qamw_stream_t stream) {
+  static const char *fn = "qamw_lloyd_assign";
+  g_last_error[0] = 0;
+  int rc;
+  if ((rc = check_lloyd(points, T, centroids, N, fn))) return rc;
+  if (!idx_inout) return fail(QAMW_ENULL, "%s: idx_inout must be non-NULL", fn);
+  cudaError_t e = launch_lloyd_assign(points, T, centroids, N, idx_inout, changed, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+int qamw_lloyd_update(const double *points, int64_t T, const int32_t *idx, int32_t N, double *centroids_inout,
+                      void *workspace, size_t workspace_bytes, qamw_stream_t stream) {
+  static const char *fn = "qamw_lloyd_update";
+  g_last_error[0] = 0;
+  int rc;
+  if ((rc = check_lloyd(points, T, centroids_inout, N, fn))) return rc;
+  if (!idx) return fail(QAMW_ENULL, "%s: idx must be non-NULL", fn);
+  const size_t need = qamw_lloyd_workspace_bytes(T, N);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(QAMW_EWORKSPACE, "%s: workspace of %zu bytes needed (got %zu)", fn, need, workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(QAMW_EINVAL, "%s: workspace must be 256-byte aligned", fn);
+  cudaError_t e = launch_lloyd_update(points, T, idx, N, centroids_inout, workspace, nullptr, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+int qamw_lloyd_train(const double *points, int64_t T, double *centroids, int32_t N, int32_t max_iter,
+                     int32_t *idx_out, void *workspace, size_t workspace_bytes, int32_t *iterations_out,
+                     int32_t *converged_out, qamw_stream_t stream) {
+  static const char *fn = "qamw_lloyd_train";
+  g_last_error[0] = 0;
+  int rc;
+  if ((rc = check_lloyd(points, T, centroids, N, fn))) return rc;
+  if (!idx_out) return fail(QAMW_ENULL, "%s: idx_out must be non-NULL", fn);
+  if (max_iter < 0) return fail(QAMW_EINVAL, "%s: max_iter (%d) must be >= 0", fn, max_iter);
+  const size_t need = qamw_lloyd_workspace_bytes(T, N);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(QAMW_EWORKSPACE, "%s: workspace of %zu bytes needed (got %zu)", fn, need, workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(QAMW_EINVAL, "%s: workspace must be 256-byte aligned", fn);
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  unsigned long long *changed = reinterpret_cast<unsigned long long *>(ws + need - 256);
+  cudaError_t e;
+  // idx = assign(C0) (every sample counts as changed: idx starts at -1)
+  if ((e = cudaMemsetAsync(idx_out, 0xff, (size_t)T * sizeof(int32_t), st)) != cudaSuccess) return cuda_fail(e, fn);
+  if ((e = launch_lloyd_assign(points, T, centroids, N, idx_out, nullptr, st)) != cudaSuccess) return cuda_fail(e, fn);
+  int32_t it = 0, conv = 0;
+  for (it = 1; it <= max_iter; ++it) {
+    if ((e = launch_lloyd_update(points, T, idx_out, N, centroids, workspace, nullptr, st)) != cudaSuccess)
+      return cuda_fail(e, fn);
+    if ((e = cudaMemsetAsync(changed, 0, sizeof(unsigned long long), st)) != cudaSuccess) return cuda_fail(e, fn);
+    if ((e = launch_lloyd_assign(points, T, centroids, N, idx_out, changed, st)) != cudaSuccess)
+      return cuda_fail(e, fn);
+    unsigned long long h = 0;
+    if ((e = cudaMemcpyAsync(&h, changed, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+      return cuda_fail(e, fn);
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, fn);
+    if (h == 0) {
+      conv = 1;
+      break;
+    }
+  }
+  if (it > max_iter) it = max_iter;
+  if (iterations_out) *iterations_out = it;
+  if (converged_out) *converged_out = conv;
+  return QAMW_OK;
+}
+
 }  // extern "C"

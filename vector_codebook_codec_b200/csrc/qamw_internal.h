@@ -125,6 +125,14 @@ bool decode_tma_applicable(const DecodeArgs &a);
 cudaError_t launch_decode_tma(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_rotate_test(const RotateTestArgs &a, cudaStream_t s);
 
+// Lloyd training of the 2D codebook (qamw_lloyd.cu); points and centroids are
+// fp64 [.][2], 16-byte aligned.
+size_t lloyd_workspace_bytes(int64_t T, int N);
+cudaError_t launch_lloyd_assign(const double *pts, int64_t T, const double *cent, int N, int32_t *idx,
+                                unsigned long long *changed, cudaStream_t s);
+cudaError_t launch_lloyd_update(const double *pts, int64_t T, const int32_t *idx, int N, double *cent,
+                                void *workspace, int32_t *empty_count, cudaStream_t s);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
