@@ -51,11 +51,12 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="llama7b_attn",
-                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4", "lloyd"),
+                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4", "lloyd", "polar"),
                    help="llama7b_attn: 4096x4096 bf16 at 2048 centroids (5.5 bits/weight; the default); "
                         "rate35 / rate4: the same matrix at 128 / 256 centroids (3.5 / 4 bits/weight); "
                         "decode_13b: decode-only sweep over the 13B shapes; tiny: 256x512 fp32; "
-                        "lloyd: codebook training, one Lloyd iteration of 2048 centroids on 2^21 samples per step")
+                        "lloyd: codebook training, one Lloyd iteration of 2048 centroids on 2^21 samples per step; "
+                        "polar: the polar baseline codec on the 4096x4096 projection at 2048 points")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
@@ -453,7 +454,113 @@ def run_lloyd(args):
     return 0
 
 
+def run_polar(args):
+    """Steps of the polar baseline codec on the 4096x4096 projection at 2048
+    points (32 amplitude levels x 64 sectors): qamw_calibrate_sigma +
+    qamw_encode_polar + qamw_decode (the polar points as codebook). Also
+    reports the whole-matrix relative error of the joint and the polar codec."""
+    import torch
+    import synth
+    import vector_codebook_codec_b200 as q
+    from vector_codebook_codec_b200 import build as qbuild
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qbuild.build()
+    spec = synth.llama7b_attn().specs[0]
+    M, K = spec.M, spec.K
+    Wt, W32 = synth.to_bf16(synth.make_matrix(spec))
+    act = synth.act_for(spec)
+    Wd, actd = Wt.to(dev), torch.from_numpy(act).to(dev)
+    pol = q.load_polar(spec.N)
+    amps = torch.from_numpy(pol["amps"]).to(dev)
+    pts = torch.from_numpy(pol["points"]).to(dev)
+    lib = q.load_library()
+    ws = torch.empty(int(lib.qamw_calibrate_workspace_bytes(M, K)), dtype=torch.uint8, device=dev)
+    wpr = q.words_per_row(K, spec.bits)
+    sigma = torch.empty(K // 2, dtype=torch.float32, device=dev)
+    packed = torch.empty((M, wpr), dtype=torch.int32, device=dev)
+    rnorm = torch.empty(M, dtype=torch.float32, device=dev)
+    cscale = torch.empty(K, dtype=torch.float32, device=dev)
+    out = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def one(evs=None):
+        if evs: evs[0].record(stream)
+        sig = q.calibrate_sigma(Wd, actd, spec.alpha, spec.block, spec.seed, status=status, workspace=ws, out=sigma)
+        if evs: evs[1].record(stream)
+        enc = q.encode_polar(Wd, actd, spec.alpha, spec.block, spec.seed, sig, amps, pol["P"], spec.bits,
+                             status=status, out=(packed, rnorm, cscale))
+        if evs: evs[2].record(stream)
+        q.decode(enc, pts, out_dtype=torch.bfloat16, status=status, out=out)
+        if evs: evs[3].record(stream)
+        return enc
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        one()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        one(ev[i])
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()}")
+    t = {k: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
+         for j, k in enumerate(("calibrate", "encode", "decode"))}
+    step_ms = sum(ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)) / args.steps
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    enc_bytes = M * K * 2 + M * wpr * 4
+    roof = {"bound": "hbm", "achieved": enc_bytes / (t["encode"] * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": enc_bytes / (t["encode"] * 1e-3) / 1e9 / hbm, "traffic": None,
+            "kernel": "encode_polar_kernel (fp64 hypot / atan2 per pair; events span the qamw_encode_polar call)",
+            "peak_source": f"{peak_kind} hbm_gbs"}
+    # quality at equal rate: whole-matrix relative error of both codecs (fp32 decode)
+    enc = one()
+    wp = q.decode(enc, pts, out_dtype=torch.float32)
+    C = torch.from_numpy(q.load_codebook(spec.N)).to(dev)
+    joint = q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sigma, C, spec.bits,
+                     search_table=q.build_search_table(C))
+    wj = q.decode(joint, C, out_dtype=torch.float32)
+    Wf = Wd.float()
+    nrm = torch.sum(Wf * Wf).item()
+    err = {"joint": torch.sum((wj - Wf) ** 2).item() / nrm, "polar": torch.sum((wp - Wf) ** 2).item() / nrm}
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import codec
+        rows = 64
+        sig_h = sigma.cpu().numpy()
+        t0 = time.perf_counter()
+        codec.encode_polar(W32[:rows], act, spec.alpha, spec.block, spec.seed, sig_h, pol["amps"], pol["P"],
+                           spec.bits)
+        dt = time.perf_counter() - t0
+        cpu = {"value": rows * K / dt / 1e9, "unit": "Gweights/s", "cores": 1, "kind": "oracle",
+               "sample": f"polar encode of {rows} of {M} rows (fp64 numpy)"}
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": M * K / (step_ms * 1e-3) / 1e9, "unit": "Gweights/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; no checkpoint)",
+            "config": {"workload": "polar_4096x4096_bf16_b128_A32xP64", "codec": "polar baseline",
+                       "A": int(amps.numel()), "P": pol["P"], "bits": spec.bits,
+                       "l2": "flushed by a 256 MiB write before every timed step"},
+            "roofline": roof, "ms": t, "relative_sq_error": err, "cpu_baseline": cpu,
+            "gpu_launches": 8 * args.steps, "clocks": clk}), flush=True)
+    return 0
+
+
 def run_ours(args):
+    if args.workload == "polar":
+        return run_polar(args)
     if args.workload == "decode_13b":
         return run_decode_sweep(args)
     if args.workload == "lloyd":

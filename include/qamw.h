@@ -192,6 +192,26 @@ int qamw_build_search_table(const float *codebook, int32_t N, void *table, size_
                             qamw_stream_t stream);
 
 /*
+ * qamw_encode_polar -- the polar baseline codec ("Joint 2D vs. Polar", Results
+ * of the QAM-W page): steps (5), (1), (2), (3) exactly as qamw_encode, then
+ * the amplitude and the phase of each normalised pair are quantized
+ * independently, at the rate of a joint codebook of A*P points:
+ *   a = number of edges (amps[i] + amps[i+1]) / 2 below hypot(x0, x1),
+ *   p = floor((atan2(x1, x0) mod 2 pi) / (2 pi / P)) mod P,  index = a * P + p,
+ * decided in fp64 from the fp32 pair. The stream decodes with qamw_decode
+ * given the A*P reconstruction points amps[a] * (cos, sin)(2 pi (p + 1/2) / P),
+ * in index order, as the codebook.
+ *   amps: device float64 [A], ascending, 8-byte aligned; 1 <= A*P <= 2^bits.
+ * Other arguments as qamw_encode (block <= 512; larger blocks return
+ * QAMW_EUNSUPPORTED).
+ */
+int qamw_encode_polar(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                      const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                      const float *sigma, const double *amps, int32_t A, int32_t P, int32_t bits_per_pair,
+                      uint32_t *packed_out, float *row_norm_out, float *col_scale_out, int32_t *status,
+                      qamw_stream_t stream);
+
+/*
  * qamw_decode -- Methodology (6) Decoding.
  * w_hat_ij = r_i * d_j * (H_b (sigma (.) C[idx]))_j / (sqrt(b) * s_j): unpack,
  * look up centroids, rescale by sigma_k, inverse rotation, multiply by the

@@ -310,3 +310,19 @@ def decode_with_scale(idx, r, sigma, s, K, block, seed, C) -> np.ndarray:
     Uh = rotate_inv(Yh, sign_mask(seed, K), block)
     s64 = np.ones(K) if s is None else np.asarray(s, dtype=np.float32).astype(np.float64)
     return Uh * np.asarray(r, dtype=np.float32).astype(np.float64)[:, None] / s64[None, :]
+
+
+def encode_polar(W, act_rms, alpha, block, seed, sigma, amps, P, bits):
+    """The polar baseline codec of "Joint 2D vs. Polar" (QAM-W page, Results):
+    steps (5), (1), (2), (3) as in :func:`encode`, then each normalised pair is
+    quantized by amplitude (nearest of the levels ``amps``) and phase (P
+    uniform sectors) independently; the index is a*P + p (the order of
+    ``PolarCode.points()``). Returns dict(packed, r, idx, margin, x, s)."""
+    from oracle.lloyd import PolarCode
+    code = PolarCode(np.asarray(amps, dtype=np.float64), P)
+    s, r, Y = rotated_rows(W, act_rms, alpha, block, seed)
+    X = normalised_pairs(Y, sigma)
+    M, Pp = X.shape[0], X.shape[1]
+    idx, margin = code.indices(X.reshape(-1, 2).astype(np.float64))
+    idx = idx.reshape(M, Pp)
+    return {"packed": pack_indices(idx, bits), "r": r, "idx": idx, "margin": margin.reshape(M, Pp), "x": X, "s": s}

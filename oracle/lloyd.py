@@ -140,6 +140,29 @@ class PolarCode:
         e = x - self.quantize(x)
         return float(np.mean(np.sum(e * e, axis=1)))
 
+    def indices(self, x: np.ndarray):
+        """Index a * P + p of each sample's reconstruction point in ``points()``
+        order (a: nearest amplitude level, p: phase sector), and the sample's
+        margin: its distance to the nearest decision boundary, relative for the
+        amplitude (|rad - edge| / rad) and in sector widths for the phase."""
+        x = np.asarray(x, dtype=np.float64)
+        rad = np.hypot(x[:, 0], x[:, 1])
+        ang = np.mod(np.arctan2(x[:, 1], x[:, 0]), 2 * math.pi)
+        w = 2 * math.pi / self.P
+        if self.amps.size > 1:
+            edges = (self.amps[1:] + self.amps[:-1]) / 2
+            ai = np.searchsorted(edges, rad)
+            lo = np.abs(rad - edges[np.maximum(ai - 1, 0)])       # the edges on either side of rad
+            hi = np.abs(edges[np.minimum(ai, edges.size - 1)] - rad)
+            near = np.minimum(lo, hi) / np.maximum(rad, 1e-300)
+        else:
+            ai = np.zeros(rad.shape, dtype=np.int64)
+            near = np.full(rad.shape, np.inf)
+        f = ang / w
+        pi_ = np.floor(f).astype(np.int64) % self.P
+        sec = np.abs(f - np.round(f)) if self.P > 1 else np.full(rad.shape, np.inf)
+        return ai * self.P + pi_, np.minimum(near, sec)
+
 
 def best_polar(samples: np.ndarray, N: int) -> PolarCode:
     """Best power-of-two split N = A*P (least MSE on ``samples``)."""

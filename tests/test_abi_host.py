@@ -158,3 +158,19 @@ def test_lloyd_entry_points_reject_on_host(lib):
                                 None) == QAMW_EINVAL
     assert lib.qamw_lloyd_train(FAKE, 10, FAKE, 4, 5, None, FAKE, ws, None, None, None) == QAMW_ENULL
     assert it.value == -5 and conv.value == -5   # untouched on a rejected call
+
+
+def test_encode_polar_rejects_on_host(lib):
+    def call(**kw):
+        a = dict(W=FAKE, wt=1, M=8, K=256, ldw=256, act=None, alpha=0.5, block=128, seed=1, sigma=FAKE,
+                 amps=FAKE, A=8, P=32, bits=8, packed=FAKE, r=FAKE, s=FAKE)
+        a.update(kw)
+        return lib.qamw_encode_polar(a["W"], a["wt"], a["M"], a["K"], a["ldw"], a["act"], a["alpha"], a["block"],
+                                     a["seed"], a["sigma"], a["amps"], a["A"], a["P"], a["bits"], a["packed"],
+                                     a["r"], a["s"], None, None)
+    assert call(amps=None) == QAMW_ENULL
+    assert call(A=0) == QAMW_EINVAL
+    assert call(P=0) == QAMW_EINVAL
+    assert call(A=16, P=32) == QAMW_EINVAL          # 512 points > 2^8
+    assert call(amps=ctypes.c_void_p(0x10004)) == QAMW_EINVAL
+    assert call(block=1024, K=1024, ldw=1024) == QAMW_EUNSUPPORTED

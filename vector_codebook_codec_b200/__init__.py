@@ -54,6 +54,8 @@ _SIGNATURES = {
     "qamw_build_search_table": (ctypes.c_int, [_c_p, _c_i32, _c_p, _c_sz, _c_p]),
     "qamw_calibrate_sigma_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
                                                     _c_i32, _c_u64, _c_p, _c_p, _c_p]),
+    "qamw_encode_polar": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32, _c_u64,
+                                         _c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p]),
     "qamw_lloyd_workspace_bytes": (_c_sz, [_c_i64, _c_i32]),
     "qamw_lloyd_assign": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_p]),
     "qamw_lloyd_update": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_sz, _c_p]),
@@ -113,6 +115,7 @@ qamw_calibrate_sigma = _raw("qamw_calibrate_sigma")
 qamw_encode = _raw("qamw_encode")
 qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
+qamw_encode_polar = _raw("qamw_encode_polar")
 qamw_lloyd_workspace_bytes = _raw("qamw_lloyd_workspace_bytes")
 qamw_lloyd_assign = _raw("qamw_lloyd_assign")
 qamw_lloyd_update = _raw("qamw_lloyd_update")
@@ -177,6 +180,15 @@ def load_codebook(N: int):
     if not os.path.exists(path):
         raise FileNotFoundError(f"no shipped codebook with N={N} ({path})")
     return np.load(path).astype(np.float32)
+
+
+def load_polar(N: int) -> dict:
+    """The shipped polar baseline code of N = A * P points: ``amps`` (float64
+    [A], ascending), ``P``, and ``points`` (float32 [N, 2], index order)."""
+    import numpy as np
+    e = codebook_manifest()[str(N)]
+    return {"amps": np.load(os.path.join(CODEBOOK_DIR, e["polar_amps_file"])), "P": int(e["polar_sectors"]),
+            "points": np.load(os.path.join(CODEBOOK_DIR, e["polar_points_file"]))}
 
 
 def codebook_manifest() -> dict:
@@ -268,6 +280,33 @@ def encode(W, act_rms, alpha: float, block: int, seed: int, sigma, codebook, bit
         _ptr(sigma), _ptr(codebook.contiguous()), N, bits, _ptr(search_table), _ptr(packed), _ptr(r), _ptr(s),
         _ptr(status), _stream_ptr(stream)))
     return Encoded(packed, r, s, sigma, M, K, block, seed, N, bits)
+
+
+def encode_polar(W, act_rms, alpha: float, block: int, seed: int, sigma, amps, P: int, bits: int,
+                 status=None, stream=None, out=None) -> Encoded:
+    """Encode W with the polar baseline code (amps: float64 CUDA tensor [A], P
+    sectors); decode the result with :func:`decode` and the code's points."""
+    torch = _torch()
+    _need_cuda("W", W, ndim=2)
+    _need_cuda("act_rms", act_rms, torch.float32, 1)
+    _need_cuda("sigma", sigma, torch.float32, 1)
+    _need_cuda("amps", amps, torch.float64, 1)
+    M, K = W.shape
+    A = amps.shape[0]
+    wpr = words_per_row(K, bits)
+    if wpr < 0:
+        raise ValueError("invalid K / bits")
+    if out is None:
+        packed = torch.empty((M, wpr), dtype=torch.int32, device=W.device)
+        r = torch.empty(M, dtype=torch.float32, device=W.device)
+        s = torch.empty(K, dtype=torch.float32, device=W.device)
+    else:
+        packed, r, s = out
+    _check("qamw_encode_polar", load_library().qamw_encode_polar(
+        _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
+        _ptr(sigma), _ptr(amps.contiguous()), A, int(P), bits, _ptr(packed), _ptr(r), _ptr(s), _ptr(status),
+        _stream_ptr(stream)))
+    return Encoded(packed, r, s, sigma, M, K, block, seed, A * int(P), bits)
 
 
 def decode(enc: Encoded, codebook, out_dtype=None, status=None, stream=None, out=None):

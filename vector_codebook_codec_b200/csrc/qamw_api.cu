@@ -201,6 +201,48 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
   return QAMW_OK;
 }
 
+int qamw_encode_polar(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                      const float *act_rms, float alpha, int32_t block, uint64_t sign_seed, const float *sigma,
+                      const double *amps, int32_t A, int32_t P, int32_t bits_per_pair, uint32_t *packed_out,
+                      float *row_norm_out, float *col_scale_out, int32_t *status, qamw_stream_t stream) {
+  static const char *fn = "qamw_encode_polar";
+  g_last_error[0] = 0;
+  int rc;
+  if (!W || !sigma || !amps || !packed_out || !row_norm_out || !col_scale_out)
+    return fail(QAMW_ENULL, "%s: W, sigma, amps, packed_out, row_norm_out, col_scale_out must be non-NULL", fn);
+  if ((rc = check_dtype(w_dtype, fn))) return rc;
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if (A < 1 || P < 1 || (int64_t)A * P > QAMW_MAX_CENTROIDS)
+    return fail(QAMW_EINVAL, "%s: A (%d) and P (%d) must be >= 1 with A*P <= %d", fn, A, P, QAMW_MAX_CENTROIDS);
+  if ((rc = check_code(A * P, bits_per_pair, fn))) return rc;
+  if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
+  if (!std::isfinite(alpha)) return fail(QAMW_EINVAL, "%s: alpha must be finite", fn);
+  if (reinterpret_cast<uintptr_t>(amps) % 8) return fail(QAMW_EINVAL, "%s: amps must be 8-byte aligned", fn);
+  if (block > 512) return fail(QAMW_EUNSUPPORTED, "%s: block %d > 512 is not supported", fn, block);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = launch_channel_scale(ScaleArgs{act_rms, alpha, K, col_scale_out, status}, st)) != cudaSuccess)
+    return cuda_fail(e, fn);
+  if ((e = launch_row_norms(RowNormArgs{W, w_dtype, M, K, ldw, col_scale_out, row_norm_out, status}, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, fn);
+  EncodeArgs ea;
+  ea.rot = RotateArgs{W, w_dtype, M, K, ldw, log2i(block), sign_seed, col_scale_out, row_norm_out};
+  ea.sigma = sigma;
+  ea.codebook = nullptr;
+  ea.N = A * P;
+  ea.bits = bits_per_pair;
+  ea.wpr = qamw_words_per_row(K, bits_per_pair);
+  ea.packed = packed_out;
+  ea.table = nullptr;
+  ea.status = status;
+  ea.polar_amps = amps;
+  ea.polar_A = A;
+  ea.polar_P = P;
+  if ((e = launch_encode_polar(ea, st)) != cudaSuccess) return cuda_fail(e, fn);
+  return QAMW_OK;
+}
+
 int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
                 int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
                 int32_t bits_per_pair, void *W_out, qamw_dtype out_dtype, int64_t ldo, int32_t *status,

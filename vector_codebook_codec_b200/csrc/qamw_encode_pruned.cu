@@ -28,31 +28,62 @@
 
 #include "qamw_device.cuh"
 #include "qamw_internal.h"
-#include "qamw_rotate16.cuh"
+#include "qamw_encode_unit.cuh"
 
 namespace qamw {
 namespace {
 
-constexpr int kWarps = kTileRows;
-constexpr int kThreads = kWarps * 32;
+constexpr int kWarps = kUnitWarps;
+constexpr int kThreads = kUnitThreads;
 
-struct ChunkTables {
-  double sd[32 * kSdPitch];       // d_j * s_j of the lane's 16 columns (0 past K)
-  double inv_sigma[32 * kIsPitch];  // 1 / sigma_k of the lane's 8 pairs (0 past K/2)
+// The exact pruned search over the codebook's grid table (see the file comment).
+struct PrunedSearch {
+  const float2 *cb2;
+  const uint16_t *toff, *lst;
+  bool use;
+  int G, N;
+  float a_ax, UL, inv_cw, Gf;
+
+  __device__ __forceinline__ void search8(const float (&x0)[8], const float (&x1)[8], int (&idx)[8]) const {
+    // candidate ranges of the 8 pairs (cell lists, or the identity list),
+    // without branches: an off-grid pair reads cell 0 and discards it
+    int beg[8], end[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const float u0 = __fdividef(x0[p], __fadd_rn(a_ax, fabsf(x0[p])));
+      const float u1 = __fdividef(x1[p], __fadd_rn(a_ax, fabsf(x1[p])));
+      const float fx = __fmul_rn(__fadd_rn(u0, UL), inv_cw);
+      const float fy = __fmul_rn(__fadd_rn(u1, UL), inv_cw);
+      const bool in = use && fx >= 0.0f && fx < Gf && fy >= 0.0f && fy < Gf;
+      const int cell = in ? (int)fy * G + (int)fx : 0;
+      const int b0 = toff[cell], e0 = toff[cell + 1];
+      beg[p] = in ? b0 : 0;
+      end[p] = in ? e0 : N;
+    }
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      float best = INFINITY;
+      int bi = 0;
+      int j = beg[p];
+      const int e = end[p];
+      for (; j < e; ++j) {
+        const int i0 = lst[j];
+        const float2 c0 = cb2[i0];
+        const float d0 = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
+        if (d0 < best) { best = d0; bi = i0; }
+      }
+      idx[p] = bi;
+    }
+  }
 };
-constexpr int kStageBytes = 512;  // per warp: 256 uint16 indices of the unit
 
 template <int WT>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_pruned_kernel(EncodeArgs a, int vec_ok, int tab_cap, int toff_slots) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const RotateArgs &ra = a.rot;
   const int N = a.N;
   const int n2 = (N + 1) & ~1;
-  ChunkTables &ct = *reinterpret_cast<ChunkTables *>(smem);
-  uint16_t *stage = reinterpret_cast<uint16_t *>(smem + sizeof(ChunkTables) + warp * kStageBytes);
-  float2 *cb2 = reinterpret_cast<float2 *>(smem + sizeof(ChunkTables) + kWarps * kStageBytes);
+  float2 *cb2 = reinterpret_cast<float2 *>(smem + kUnitSmemBytes);
   uint16_t *toff = reinterpret_cast<uint16_t *>(cb2 + n2);
   uint16_t *lst = toff + toff_slots;   // identity list 0..N-1, then the cell lists
 
@@ -89,135 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const float a_ax = s_a, UL = s_UL, inv_cw = s_inv, Gf = (float)G;
 
-  const int64_t M = ra.M, K = ra.K, P = K >> 1;
-  const int64_t n_chunks = (K + kUnit - 1) / kUnit;
-  const int64_t RG = (M + kTileRows - 1) / kTileRows;
-  const int64_t T = n_chunks * RG;
-  const int64_t t0 = (int64_t)blockIdx.x * T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
-  const double inv_sqrt_b = 1.0 / sqrt((double)(1 << ra.log2b));
-  const int B = a.bits;
-  // floor(n / B) = (n * divB) >> 32 exactly for 0 <= n < 2^14 and 1 <= B <= 16
-  // (checked exhaustively); the packing needs n < 256 * 16 + 32
-  const uint64_t divB = (0x100000000ull / (uint64_t)B) + 1ull;
-
-  // the next unit's weights and row norm, loaded while the current one is searched
-  auto prefetch = [&](int64_t t, WRegs<WT> &w, float &rn) -> bool {
-    const int64_t chunk = t / RG, row = (t % RG) * kTileRows + warp;
-    rn = 0.0f;
-    if (row >= M) return false;
-    rn = ra.r[row];
-    return load_unit16<WT>(w, ra.W, ra.ldw, K, row, chunk * kUnit + 16 * lane, vec_ok);
-  };
-
-  WRegs<WT> wn;
-  float rn_next = 0.0f;
-  bool full_next = (t0 < t1) ? prefetch(t0, wn, rn_next) : false;
-  int64_t cur_chunk = -1;
-  for (int64_t t = t0; t < t1; ++t) {
-    const int64_t chunk = t / RG, g = t % RG;
-    if (chunk != cur_chunk) {
-      __syncthreads();   // every warp is done with the previous chunk's tables (and the table copy is complete)
-      load_sd512(ct.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
-      if (threadIdx.x < kUnit / 2) {
-        // a rotated unit row has |y_j| <= 1 (to within the fp32 rounding of r),
-        // so |x| <= 1 / sigma_k: every x of the column is a finite fp32 when
-        // 1 / sigma_k is at most half the fp32 range (else the status says so)
-        const int i = threadIdx.x;
-        const int64_t p = chunk * (kUnit / 2) + i;
-        const double is = (p < P) ? 1.0 / (double)a.sigma[p] : 0.0;
-        ct.inv_sigma[(i >> 3) * kIsPitch + (i & 7)] = is;
-        if (!(fabs(is) <= 0.5 * (double)FLT_MAX)) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
-      }
-      __syncthreads();
-      cur_chunk = chunk;
-    }
-    const WRegs<WT> wc = wn;
-    const bool full = full_next;
-    const float r = rn_next;
-    if (t + 1 < t1) full_next = prefetch(t + 1, wn, rn_next);
-
-    const int64_t row = g * kTileRows + warp;
-    if (row >= M) continue;
-    const int64_t col = chunk * kUnit + 16 * lane;
-
-    float x0[8], x1[8];
-    uint32_t bad = 0;
-    if (r > 0.0f && isfinite(r)) {
-      double v[16];
-      scaled16<WT>(v, wc, full, ra.W, ra.ldw, K, row, col, &ct.sd[lane * kSdPitch]);
-      fwht16_fp64(v, ra.log2b, lane);
-      const double qn = inv_sqrt_b / (double)r;
-      const double2 *is2 = reinterpret_cast<const double2 *>(&ct.inv_sigma[lane * kIsPitch]);
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const double2 is = is2[h];
-        const double f0 = qn * is.x, f1 = qn * is.y;
-        x0[2 * h] = (float)(v[4 * h] * f0);
-        x1[2 * h] = (float)(v[4 * h + 1] * f0);
-        x0[2 * h + 1] = (float)(v[4 * h + 2] * f1);
-        x1[2 * h + 1] = (float)(v[4 * h + 3] * f1);
-      }
-    } else {
-      if (!(r == 0.0f)) bad = 1;   // NaN / Inf row norm; a zero row codes every pair as x = 0
-#pragma unroll
-      for (int p = 0; p < 8; ++p) { x0[p] = 0.0f; x1[p] = 0.0f; }
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
-
-    // candidate ranges of the 8 pairs (cell lists, or the identity list),
-    // without branches: an off-grid pair reads cell 0 and discards it
-    int beg[8], end[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      const float u0 = __fdividef(x0[p], __fadd_rn(a_ax, fabsf(x0[p])));
-      const float u1 = __fdividef(x1[p], __fadd_rn(a_ax, fabsf(x1[p])));
-      const float fx = __fmul_rn(__fadd_rn(u0, UL), inv_cw);
-      const float fy = __fmul_rn(__fadd_rn(u1, UL), inv_cw);
-      const bool in = use && fx >= 0.0f && fx < Gf && fy >= 0.0f && fy < Gf;
-      const int cell = in ? (int)fy * G + (int)fx : 0;
-      const int b0 = toff[cell], e0 = toff[cell + 1];
-      beg[p] = in ? b0 : 0;
-      end[p] = in ? e0 : N;
-    }
-    int idx[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      float best = INFINITY;
-      int bi = 0;
-      int j = beg[p];
-      const int e = end[p];
-      for (; j < e; ++j) {
-        const int i0 = lst[j];
-        const float2 c0 = cb2[i0];
-        const float d0 = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
-        if (d0 < best) { best = d0; bi = i0; }
-      }
-      idx[p] = bi;
-    }
-
-    // pack: stage the unit's 256 indices, then build the unit's words
-    __syncwarp();
-    reinterpret_cast<uint4 *>(stage)[lane] =
-        make_uint4((uint32_t)idx[0] | ((uint32_t)idx[1] << 16), (uint32_t)idx[2] | ((uint32_t)idx[3] << 16),
-                   (uint32_t)idx[4] | ((uint32_t)idx[5] << 16), (uint32_t)idx[6] | ((uint32_t)idx[7] << 16));
-    __syncwarp();
-    const int64_t pair0 = chunk * (kUnit / 2);
-    const int np = (int)((P - pair0) < (kUnit / 2) ? (P - pair0) : (kUnit / 2));
-    const int nw = (np * B + 31) >> 5;
-    uint32_t *dst = a.packed + row * a.wpr + chunk * (int64_t)(8 * B);
-    for (int w = lane; w < nw; w += 32) {
-      const int bit0 = w * 32;
-      const int k0 = (int)(((uint64_t)bit0 * divB) >> 32);               // bit0 / B
-      const int k1 = min((int)(((uint64_t)(bit0 + 31) * divB) >> 32), np - 1);
-      uint32_t word = 0;
-      for (int k = k0; k <= k1; ++k) {
-        const int off = k * B - bit0;
-        const uint32_t iv = stage[k];
-        word |= (off >= 0) ? (iv << off) : (iv >> (-off));
-      }
-      dst[w] = word;
-    }
-  }
+  const PrunedSearch S{cb2, toff, lst, use, G, N, a_ax, UL, inv_cw, Gf};
+  encode_units<WT>(a, vec_ok, smem, S);
 }
 
 template <typename Kern>
@@ -234,8 +138,7 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
   const int G = search_grid(a.N);
   const int toff_slots = (G * G + 1 + 7) & ~7;
   const int n2 = (a.N + 1) & ~1;
-  const size_t base = sizeof(ChunkTables) + (size_t)kWarps * kStageBytes + (size_t)n2 * sizeof(float2) +
-                      (size_t)toff_slots * 2;
+  const size_t base = kUnitSmemBytes + (size_t)n2 * sizeof(float2) + (size_t)toff_slots * 2;
   const int64_t room = ((int64_t)smem_max - 128 /*static*/ - (int64_t)base) / 2;
   int tab_cap = (int)std::max<int64_t>(0, std::min<int64_t>(room, 65535));
   tab_cap &= ~7;

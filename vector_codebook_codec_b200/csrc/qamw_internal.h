@@ -77,6 +77,8 @@ struct EncodeArgs {
   uint32_t *packed;      // [M][wpr]
   const void *table;     // search table or nullptr (brute force)
   int32_t *status;
+  const double *polar_amps = nullptr;   // polar baseline: A amplitude levels (ascending), P sectors
+  int32_t polar_A = 0, polar_P = 0;
 };
 
 struct DecodeArgs {
@@ -119,6 +121,8 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
 constexpr int kPrunedMaxN = 2048;
 bool encode_pruned_applicable(const EncodeArgs &a);
 cudaError_t launch_encode_pruned(const EncodeArgs &a, cudaStream_t s);
+// The polar baseline encode (qamw_encode_polar.cu), b <= 512.
+cudaError_t launch_encode_polar(const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 // bf16 decode with TMA tensor loads/stores (qamw_decode_tma.cu).
 bool decode_tma_applicable(const DecodeArgs &a);
