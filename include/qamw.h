@@ -130,7 +130,7 @@ int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K
  * workspace, using a fixed scratch area of QAMW_NOALLOC_SCRATCH_BYTES bytes
  * built into the library; neither it nor the library allocates anything.
  *   - Limit: qamw_calibrate_workspace_bytes(M, K) must not exceed
- *     QAMW_NOALLOC_SCRATCH_BYTES (about M*K <= 33.5 million weights);
+ *     QAMW_NOALLOC_SCRATCH_BYTES (about M*K <= 58 million weights);
  *     larger shapes return QAMW_EUNSUPPORTED with a message that says so.
  *   - The area is reserved on every GPU that loads the library, until the
  *     process exits.

@@ -58,7 +58,7 @@ def test_status_strings(lib):
 def test_calibrate_workspace_bytes(lib):
     M, K = 4096, 4096
     n = lib.qamw_calibrate_workspace_bytes(M, K)
-    groups = (M + 15) // 16
+    groups = (M + 27) // 28
     assert n >= groups * (K // 2) * 8 + 4 * M + 4 * K
     assert lib.qamw_calibrate_workspace_bytes(0, 8) == 0
 

@@ -2,10 +2,10 @@
 // QAM-W Codec", QAM-W Technical Summary) for Hadamard blocks b <= 512.
 //
 // sigma_k = RN32(sqrt(2/pi) * (1/M) * sum_i ||z_ik||) over the rotated unit
-// rows. A CTA of 16 warps takes a contiguous range of tiles (16 rows x one
-// 512-column chunk) in chunk-major order, warp w holding row 16g + w with the
-// 512-column unit of qamw_rotate16.cuh. The 16 rows' ||z_ik|| are added in
-// shared memory in row order (w = 0..15) and written as the row group's fp64
+// rows. A CTA of 28 warps takes a contiguous range of tiles (28 rows x one
+// 512-column chunk) in chunk-major order, warp w holding row 28g + w with the
+// 512-column unit of qamw_rotate16.cuh. The 28 rows' ||z_ik|| are added in
+// shared memory in row order (w = 0..27) and written as the row group's fp64
 // partial sum; sigma_reduce (qamw_encode.cu) adds the groups in a fixed order.
 // The sums are the same, in the same order, as those of the 1024-column
 // calibrate kernel, so both give the same sigma.
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate512_kernel(CalibArgs a, 
     const int64_t chunk = t / RG, g = t % RG;
     if (chunk != cur_chunk) {
       __syncthreads();
-      load_sd512(sm.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
+      if (threadIdx.x < kUnit) load_sd512(sm.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
       __syncthreads();
       cur_chunk = chunk;
     }

@@ -16,7 +16,7 @@
 // Task geometry: a warp decodes ROWS rows x SEGS segments of 64 columns with
 // lane = row + ROWS * segment; each lane owns one segment of one row: 32
 // indices, i.e. exactly `bits` packed words starting on a word boundary, and
-// 64 fp32 values (about 100 registers, 16 warps per SM). SEGS is the larger
+// 64 fp32 values (128 registers, 16 warps per SM). SEGS is the larger
 // of b/64 (the lanes of one block) and the segments whose words make a
 // multiple of 16 bytes (a TMA box row must): 1 for bits % 4 == 0, 2 for even
 // bits, 4 for odd bits. Block bits 1..5 are butterflies inside the lane, bits

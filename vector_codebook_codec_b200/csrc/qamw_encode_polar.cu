@@ -66,7 +66,7 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(encode_polar_kernel<WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t n_chunks = (a.rot.K + kUnit - 1) / kUnit;
-  const int64_t tiles = n_chunks * ((a.rot.M + kTileRows - 1) / kTileRows);
+  const int64_t tiles = n_chunks * ((a.rot.M + kUnitWarps - 1) / kUnitWarps);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count()));
   const size_t es = (WT == QAMW_BF16) ? 2 : 4;
   const int vec = ((reinterpret_cast<uintptr_t>(a.rot.W) % 16) == 0 && (a.rot.ldw * (int64_t)es) % 16 == 0) ? 1 : 0;

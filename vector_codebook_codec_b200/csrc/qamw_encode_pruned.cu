@@ -10,8 +10,8 @@
 // Work decomposition. A *unit* is one row x 512 consecutive columns handled by
 // one warp: lane l owns columns [16l, 16l + 16) of the unit (8 pairs); the
 // rotation is the fp64 one of qamw_rotate16.cuh, which gives the same x bit
-// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 16 warps takes a contiguous
-// range of *tiles* (16 rows x one 512-column chunk) in chunk-major order; the
+// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 28 warps takes a contiguous
+// range of *tiles* (28 rows x one 512-column chunk) in chunk-major order; the
 // chunk's d_j * s_j and 1 / sigma_k live once per CTA in shared memory, next
 // to the codebook and the search table. The next unit's weights are loaded
 // while the current one is searched.
@@ -33,7 +33,6 @@
 namespace qamw {
 namespace {
 
-constexpr int kWarps = kUnitWarps;
 constexpr int kThreads = kUnitThreads;
 
 // The exact pruned search over the codebook's grid table (see the file comment).
@@ -146,7 +145,7 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
   const size_t smem = base + (size_t)tab_cap * 2;
   if ((e = set_smem(encode_pruned_kernel<WT>, smem)) != cudaSuccess) return e;
   const int64_t n_chunks = (a.rot.K + kUnit - 1) / kUnit;
-  const int64_t tiles = n_chunks * ((a.rot.M + kTileRows - 1) / kTileRows);
+  const int64_t tiles = n_chunks * ((a.rot.M + kUnitWarps - 1) / kUnitWarps);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count()));
   const size_t es = (WT == QAMW_BF16) ? 2 : 4;
   const int vec = ((reinterpret_cast<uintptr_t>(a.rot.W) % 16) == 0 && (a.rot.ldw * (int64_t)es) % 16 == 0) ? 1 : 0;

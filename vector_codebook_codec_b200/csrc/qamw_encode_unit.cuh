@@ -12,8 +12,8 @@
 // Work decomposition. A *unit* is one row x 512 consecutive columns handled by
 // one warp: lane l owns columns [16l, 16l + 16) of the unit (8 pairs); the
 // rotation is the fp64 one of qamw_rotate16.cuh, which gives the same x bit
-// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 16 warps takes
-// a contiguous range of *tiles* (16 rows x one 512-column chunk) in
+// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 28 warps takes
+// a contiguous range of *tiles* (one row per warp x one 512-column chunk) in
 // chunk-major order; the chunk's d_j * s_j and 1 / sigma_k live once per CTA in
 // shared memory. The next unit's weights are loaded while the current one is
 // quantized. The search policy S maps the 8 pairs (x0[p], x1[p]) of a lane to
@@ -29,7 +29,7 @@
 
 namespace qamw {
 
-constexpr int kUnitWarps = kTileRows;
+constexpr int kUnitWarps = 28;  // warps per CTA = rows per tile; 4096^2 encode: 16 warps 146 us, 20 137, 24 132, 28 126
 constexpr int kUnitThreads = kUnitWarps * 32;
 
 struct ChunkTables {
@@ -49,7 +49,7 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
   uint16_t *stage = reinterpret_cast<uint16_t *>(smem + sizeof(ChunkTables) + warp * kStageBytes);
   const int64_t M = ra.M, K = ra.K, P = K >> 1;
   const int64_t n_chunks = (K + kUnit - 1) / kUnit;
-  const int64_t RG = (M + kTileRows - 1) / kTileRows;
+  const int64_t RG = (M + kUnitWarps - 1) / kUnitWarps;
   const int64_t T = n_chunks * RG;
   const int64_t t0 = (int64_t)blockIdx.x * T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
   const double inv_sqrt_b = 1.0 / sqrt((double)(1 << ra.log2b));
@@ -60,7 +60,7 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
 
   // the next unit's weights and row norm, loaded while the current one is searched
   auto prefetch = [&](int64_t t, WRegs<WT> &w, float &rn) -> bool {
-    const int64_t chunk = t / RG, row = (t % RG) * kTileRows + warp;
+    const int64_t chunk = t / RG, row = (t % RG) * kUnitWarps + warp;
     rn = 0.0f;
     if (row >= M) return false;
     rn = ra.r[row];
@@ -75,7 +75,7 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
     const int64_t chunk = t / RG, g = t % RG;
     if (chunk != cur_chunk) {
       __syncthreads();   // every warp is done with the previous chunk's tables (and the table copy is complete)
-      load_sd512(ct.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
+      if (threadIdx.x < kUnit) load_sd512(ct.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
       if (threadIdx.x < kUnit / 2) {
         // a rotated unit row has |y_j| <= 1 (to within the fp32 rounding of r),
         // so |x| <= 1 / sigma_k: every x of the column is a finite fp32 when
@@ -94,7 +94,7 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
     const float r = rn_next;
     if (t + 1 < t1) full_next = prefetch(t + 1, wn, rn_next);
 
-    const int64_t row = g * kTileRows + warp;
+    const int64_t row = g * kUnitWarps + warp;
     if (row >= M) continue;
     const int64_t col = chunk * kUnit + 16 * lane;
 

@@ -12,7 +12,7 @@ namespace qamw {
 
 // Rows per calibration row group (fixed, so the fp64 reduction order -- and
 // hence sigma -- does not depend on the device or the grid size).
-constexpr int kCalibRowGroup = 16;
+constexpr int kCalibRowGroup = 28;
 // Columns handled by one warp in the encode / calibrate kernels (32 lanes x 32).
 constexpr int kUnitCols = 1024;
 

@@ -18,7 +18,7 @@
 namespace qamw {
 
 constexpr int kUnit = 512;        // columns per unit
-constexpr int kTileRows = 16;     // rows per tile: one per warp of a 512-thread CTA
+constexpr int kTileRows = 28;     // calibration rows per tile: one per warp (896-thread CTA; 28 measured fastest)
 constexpr int kSdPitch = 18;      // doubles per lane row of a d_j s_j table: 16 used (144-byte rows keep 16-byte loads conflict-free)
 constexpr int kIsPitch = 10;      // doubles per lane row of a per-pair table: 8 used (80-byte rows)
 
