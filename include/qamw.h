@@ -241,6 +241,17 @@ int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t b
                      uint64_t sign_seed, int32_t inverse, qamw_stream_t stream);
 
 /*
+ * qamw_selftest_wait_timeout -- test hook for failure detection (an interface
+ * of this library; the QAM-W page has no counterpart). Launches one warp that
+ * waits, with the bounded mbarrier wait the TMA decode uses (at most `tries`
+ * attempts), on a barrier no one arrives on; when the wait runs out it sets
+ * QAMW_STATUS_TIMEOUT in *status (device int32) and returns. Nothing hangs or
+ * faults; the context stays usable.
+ * Errors: QAMW_ENULL (status), QAMW_EINVAL (tries not in [1, 2^20]).
+ */
+int qamw_selftest_wait_timeout(uint32_t tries, int32_t *status, qamw_stream_t stream);
+
+/*
  * Lloyd training of the 2D codebook -- Methodology (4) Joint 2D Quantization
  * and "Significance and Claims" (the codebook is a 2D Lloyd-Max quantizer
  * trained once on samples of the unit circular Gaussian). One iteration:

@@ -174,3 +174,9 @@ def test_encode_polar_rejects_on_host(lib):
     assert call(A=16, P=32) == QAMW_EINVAL          # 512 points > 2^8
     assert call(amps=ctypes.c_void_p(0x10004)) == QAMW_EINVAL
     assert call(block=1024, K=1024, ldw=1024) == QAMW_EUNSUPPORTED
+
+
+def test_selftest_rejects_on_host(lib):
+    assert lib.qamw_selftest_wait_timeout(5, None, None) == QAMW_ENULL
+    assert lib.qamw_selftest_wait_timeout(0, FAKE, None) == QAMW_EINVAL
+    assert lib.qamw_selftest_wait_timeout((1 << 20) + 1, FAKE, None) == QAMW_EINVAL

@@ -56,6 +56,7 @@ _SIGNATURES = {
                                                     _c_i32, _c_u64, _c_p, _c_p, _c_p]),
     "qamw_encode_polar": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32, _c_u64,
                                          _c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    "qamw_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _c_p, _c_p]),
     "qamw_lloyd_workspace_bytes": (_c_sz, [_c_i64, _c_i32]),
     "qamw_lloyd_assign": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_p]),
     "qamw_lloyd_update": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_sz, _c_p]),
@@ -116,6 +117,7 @@ qamw_encode = _raw("qamw_encode")
 qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
 qamw_encode_polar = _raw("qamw_encode_polar")
+qamw_selftest_wait_timeout = _raw("qamw_selftest_wait_timeout")
 qamw_lloyd_workspace_bytes = _raw("qamw_lloyd_workspace_bytes")
 qamw_lloyd_assign = _raw("qamw_lloyd_assign")
 qamw_lloyd_update = _raw("qamw_lloyd_update")
@@ -393,3 +395,51 @@ def lloyd_train(points, init, max_iter: int = 500, stream=None):
         _ptr(points), T, _ptr(C), N, int(max_iter), _ptr(idx), _ptr(ws), need, ctypes.byref(it),
         ctypes.byref(conv), _stream_ptr(stream)))
     return C, idx, int(it.value), bool(conv.value)
+
+
+# ---------------------------------------------------------------------------
+# the encoded artefact on disk
+# ---------------------------------------------------------------------------
+
+ENCODED_FORMAT = "qamw-encoded"
+ENCODED_VERSION = 1
+
+
+def save_encoded(path: str, enc: Encoded, codebook) -> None:
+    """Writes an encoded matrix and its codebook to ``path`` (numpy .npz): the
+    packed words, r_i, s_j, sigma_k, the codebook, and block, seed, N, bits,
+    M, K, with a format name and version. Everything qamw_decode needs."""
+    import numpy as np
+
+    def host(t):
+        return t.detach().cpu().numpy() if hasattr(t, "detach") else np.asarray(t)
+
+    np.savez(path, format=np.array(ENCODED_FORMAT), version=np.array(ENCODED_VERSION, dtype=np.int32),
+             packed=host(enc.packed).view(np.uint32), row_norm=host(enc.row_norm).astype(np.float32),
+             col_scale=host(enc.col_scale).astype(np.float32), sigma=host(enc.sigma).astype(np.float32),
+             codebook=host(codebook).astype(np.float32),
+             shape=np.array([enc.M, enc.K, enc.block, enc.N, enc.bits], dtype=np.int64),
+             seed=np.array(enc.seed, dtype=np.uint64))
+
+
+def load_encoded(path: str, device="cuda"):
+    """Reads a file written by :func:`save_encoded`; returns (Encoded, codebook)
+    as tensors on ``device``. Raises ValueError on another format or version."""
+    import numpy as np
+    torch = _torch()
+    with np.load(path, allow_pickle=False) as z:
+        if str(z["format"]) != ENCODED_FORMAT:
+            raise ValueError(f"{path}: not a {ENCODED_FORMAT} file")
+        if int(z["version"]) != ENCODED_VERSION:
+            raise ValueError(f"{path}: format version {int(z['version'])}, expected {ENCODED_VERSION}")
+        M, K, block, N, bits = (int(v) for v in z["shape"])
+        seed = int(z["seed"])
+        if words_per_row(K, bits) != z["packed"].shape[1] or z["packed"].shape[0] != M:
+            raise ValueError(f"{path}: packed words do not match M, K, bits")
+
+        def dev(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+        enc = Encoded(dev(z["packed"].view(np.int32)), dev(z["row_norm"]), dev(z["col_scale"]), dev(z["sigma"]),
+                      M, K, block, seed, N, bits)
+        return enc, dev(z["codebook"])

@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "qamw.h"
 #include "qamw_internal.h"
 
@@ -37,6 +39,15 @@ int log2i(int64_t v) {
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// An NVTX range around one C-ABI call (visible to nsys / ncu when attached;
+// a few nanoseconds otherwise).
+struct CallRange {
+  explicit CallRange(const char *name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange &) = delete;
+  CallRange &operator=(const CallRange &) = delete;
+};
 
 // Shape checks common to calibrate / encode / decode.
 int check_shape(int64_t M, int64_t K, int32_t block, const char *fn) {
@@ -133,6 +144,7 @@ int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K
                          float *sigma_out, void *workspace, size_t workspace_bytes, int32_t *status,
                          qamw_stream_t stream) {
   static const char *fn = "qamw_calibrate_sigma";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if (W == nullptr || sigma_out == nullptr) return fail(QAMW_ENULL, "%s: W and sigma_out must be non-NULL", fn);
@@ -169,6 +181,7 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
                 const void *search_table, uint32_t *packed_out, float *row_norm_out,
                 float *col_scale_out, int32_t *status, qamw_stream_t stream) {
   static const char *fn = "qamw_encode";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if (!W || !sigma || !codebook || !packed_out || !row_norm_out || !col_scale_out)
@@ -206,6 +219,7 @@ int qamw_encode_polar(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, i
                       const double *amps, int32_t A, int32_t P, int32_t bits_per_pair, uint32_t *packed_out,
                       float *row_norm_out, float *col_scale_out, int32_t *status, qamw_stream_t stream) {
   static const char *fn = "qamw_encode_polar";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if (!W || !sigma || !amps || !packed_out || !row_norm_out || !col_scale_out)
@@ -248,6 +262,7 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
                 int32_t bits_per_pair, void *W_out, qamw_dtype out_dtype, int64_t ldo, int32_t *status,
                 qamw_stream_t stream) {
   static const char *fn = "qamw_decode";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if (!packed || !row_norm || !sigma || !codebook || !W_out)
@@ -285,6 +300,7 @@ size_t qamw_search_table_bytes(int32_t N) {
 int qamw_build_search_table(const float *codebook, int32_t N, void *table, size_t table_bytes,
                             qamw_stream_t stream) {
   static const char *fn = "qamw_build_search_table";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   if (!codebook || !table) return fail(QAMW_ENULL, "%s: codebook and table must be non-NULL", fn);
   if (N < 1) return fail(QAMW_EINVAL, "%s: N must be >= 1 (got %d)", fn, N);
@@ -299,6 +315,7 @@ int qamw_build_search_table(const float *codebook, int32_t N, void *table, size_
 int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t block, uint64_t sign_seed,
                      int32_t inverse, qamw_stream_t stream) {
   static const char *fn = "qamw_rotate_rows";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if (!U || !Y) return fail(QAMW_ENULL, "%s: U and Y must be non-NULL", fn);
@@ -326,6 +343,7 @@ static int check_lloyd(const void *points, int64_t T, const void *centroids, int
 int qamw_lloyd_assign(const double *points, int64_t T, const double *centroids, int32_t N, int32_t *idx_inout,
                       unsigned long long *changed, qamw_stream_t stream) {
   static const char *fn = "qamw_lloyd_assign";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if ((rc = check_lloyd(points, T, centroids, N, fn))) return rc;
@@ -337,6 +355,7 @@ int qamw_lloyd_assign(const double *points, int64_t T, const double *centroids, 
 int qamw_lloyd_update(const double *points, int64_t T, const int32_t *idx, int32_t N, double *centroids_inout,
                       void *workspace, size_t workspace_bytes, qamw_stream_t stream) {
   static const char *fn = "qamw_lloyd_update";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if ((rc = check_lloyd(points, T, centroids_inout, N, fn))) return rc;
@@ -353,6 +372,7 @@ int qamw_lloyd_train(const double *points, int64_t T, double *centroids, int32_t
                      int32_t *idx_out, void *workspace, size_t workspace_bytes, int32_t *iterations_out,
                      int32_t *converged_out, qamw_stream_t stream) {
   static const char *fn = "qamw_lloyd_train";
+  CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
   if ((rc = check_lloyd(points, T, centroids, N, fn))) return rc;
@@ -389,6 +409,16 @@ int qamw_lloyd_train(const double *points, int64_t T, double *centroids, int32_t
   if (iterations_out) *iterations_out = it;
   if (converged_out) *converged_out = conv;
   return QAMW_OK;
+}
+
+int qamw_selftest_wait_timeout(uint32_t tries, int32_t *status, qamw_stream_t stream) {
+  static const char *fn = "qamw_selftest_wait_timeout";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  if (status == nullptr) return fail(QAMW_ENULL, "%s: status must be non-NULL", fn);
+  if (tries < 1 || tries > (1u << 20)) return fail(QAMW_EINVAL, "%s: tries (%u) must be in [1, 2^20]", fn, tries);
+  cudaError_t e = launch_wait_timeout(tries, status, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
 }
 
 }  // extern "C"

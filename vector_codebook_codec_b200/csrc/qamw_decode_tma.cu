@@ -34,6 +34,7 @@
 
 #include "qamw_device.cuh"
 #include "qamw_internal.h"
+#include "qamw_mbarrier.cuh"
 
 namespace qamw {
 namespace {
@@ -42,31 +43,6 @@ constexpr int kSeg = 64;
 constexpr int kMaxWarps = 16;
 constexpr uint32_t kWaitLimit = 1u << 22;   // try_wait attempts before giving up
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait; returns false if the phase did not complete in time.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
-}
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -279,7 +255,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
       __syncwarp();
       cur = segcol;
     }
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], parity))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[st], parity, kWaitLimit))) {
       timed_out = true;
       break;
     }

@@ -137,6 +137,9 @@ cudaError_t launch_lloyd_assign(const double *pts, int64_t T, const double *cent
 cudaError_t launch_lloyd_update(const double *pts, int64_t T, const int32_t *idx, int N, double *cent,
                                 void *workspace, int32_t *empty_count, cudaStream_t s);
 
+// Test hook: a bounded wait on an mbarrier that never completes (qamw_selftest.cu).
+cudaError_t launch_wait_timeout(uint32_t tries, int32_t *status, cudaStream_t s);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
