@@ -118,6 +118,30 @@ int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K
                          int32_t *status, qamw_stream_t stream);
 
 /*
+ * qamw_calibrate_partial_sums / qamw_sigma_from_partial_sums -- the calibration
+ * of one matrix whose rows are split across devices (or calls). sigma_k is a
+ * mean over all M rows, so each shard of rows contributes its sum of |z_ik|
+ * (Methodology (3)); the shards' sums are exchanged (one all-gather) and
+ * combined:
+ *   qamw_calibrate_partial_sums: sums_out[k] = sum over the shard's rows i of
+ *     |z_ik| in fp64, in the fixed order qamw_calibrate_sigma uses (same
+ *     arguments and workspace as qamw_calibrate_sigma; sums_out: device
+ *     float64 [K/2]);
+ *   qamw_sigma_from_partial_sums: sums = device float64 [R][P] (shard r's sums
+ *     in row r), added in shard order; sigma_out[k] = RN32(sqrt(2/pi) *
+ *     total_k / M_total), 0 -> 1.
+ * With one shard (R = 1, M_total = M) the result equals qamw_calibrate_sigma's
+ * bit for bit. Errors: as qamw_calibrate_sigma; QAMW_EINVAL for R, P or
+ * M_total < 1.
+ */
+int qamw_calibrate_partial_sums(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                                const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                                double *sums_out, void *workspace, size_t workspace_bytes, int32_t *status,
+                                qamw_stream_t stream);
+int qamw_sigma_from_partial_sums(const double *sums, int32_t R, int64_t P, int64_t M_total, float *sigma_out,
+                                 qamw_stream_t stream);
+
+/*
  * qamw_calibrate_sigma_noalloc -- qamw_calibrate_sigma for callers that cannot
  * allocate device memory.
  * (An interface of this library; the QAM-W page has no counterpart.)

@@ -180,3 +180,13 @@ def test_selftest_rejects_on_host(lib):
     assert lib.qamw_selftest_wait_timeout(5, None, None) == QAMW_ENULL
     assert lib.qamw_selftest_wait_timeout(0, FAKE, None) == QAMW_EINVAL
     assert lib.qamw_selftest_wait_timeout((1 << 20) + 1, FAKE, None) == QAMW_EINVAL
+
+
+def test_sharded_calibration_rejects_on_host(lib):
+    assert lib.qamw_sigma_from_partial_sums(None, 1, 8, 8, FAKE, None) == QAMW_ENULL
+    assert lib.qamw_sigma_from_partial_sums(FAKE, 0, 8, 8, FAKE, None) == QAMW_EINVAL
+    assert lib.qamw_sigma_from_partial_sums(FAKE, 1, 8, 0, FAKE, None) == QAMW_EINVAL
+    assert lib.qamw_calibrate_partial_sums(FAKE, 1, 8, 256, 256, None, 0.5, 128, 1, None, FAKE, 1 << 30, None,
+                                           None) == QAMW_ENULL
+    assert lib.qamw_calibrate_partial_sums(FAKE, 1, 8, 256, 256, None, 0.5, 128, 1, FAKE, None, 0, None,
+                                           None) == QAMW_EWORKSPACE

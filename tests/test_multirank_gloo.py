@@ -56,3 +56,56 @@ def test_single_rank_helpers_without_process_group():
     import bench
     assert bench.max_over_ranks(3.0) == 3.0
     assert bench.aggregate_throughput(10.0, 2.0, 1) == 5.0
+
+
+def _shard_worker(rank, world, port, q):
+    """Row-sharded calibration, exchange step: every rank holds the fp64 sums
+    of |z| over its rows; gather_partial_sums must give every rank all of them
+    in rank order (the sums here come from the oracle's rotation: no GPU)."""
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import vector_codebook_codec_b200 as qamw
+    from oracle import codec
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    spec = synth.tiny().specs[0]
+    W = synth.make_matrix(spec)
+    act = synth.act_for(spec)
+    bounds = [0, 100, spec.M]                     # uneven shards
+    lo, hi = bounds[rank], bounds[rank + 1]
+    _, _, Y = codec.rotated_rows(W[lo:hi], act, spec.alpha, spec.block, spec.seed)
+    mine = np.sqrt(np.sum(codec.pairs(Y) ** 2, axis=2)).sum(axis=0)
+    got = qamw.gather_partial_sums(torch.from_numpy(mine))
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, got.numpy()))
+
+
+def test_sharded_calibration_exchange_gloo():
+    import numpy as np
+
+    import synth
+    from oracle import codec
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    spec = synth.tiny().specs[0]
+    W = synth.make_matrix(spec)
+    act = synth.act_for(spec)
+    _, _, Y = codec.rotated_rows(W, act, spec.alpha, spec.block, spec.seed)
+    whole = np.sqrt(np.sum(codec.pairs(Y) ** 2, axis=2)).sum(axis=0)
+    assert res[0].shape == (2, spec.K // 2)
+    assert np.array_equal(res[0], res[1])                     # every rank has the same table
+    assert np.allclose(res[0][0] + res[0][1], whole, rtol=1e-12, atol=0)

@@ -57,6 +57,9 @@ _SIGNATURES = {
     "qamw_encode_polar": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32, _c_u64,
                                          _c_p, _c_p, _c_i32, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p]),
     "qamw_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _c_p, _c_p]),
+    "qamw_calibrate_partial_sums": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
+                                                   _c_i32, _c_u64, _c_p, _c_p, _c_sz, _c_p, _c_p]),
+    "qamw_sigma_from_partial_sums": (ctypes.c_int, [_c_p, _c_i32, _c_i64, _c_i64, _c_p, _c_p]),
     "qamw_lloyd_workspace_bytes": (_c_sz, [_c_i64, _c_i32]),
     "qamw_lloyd_assign": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_p]),
     "qamw_lloyd_update": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_i32, _c_p, _c_p, _c_sz, _c_p]),
@@ -118,6 +121,8 @@ qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
 qamw_encode_polar = _raw("qamw_encode_polar")
 qamw_selftest_wait_timeout = _raw("qamw_selftest_wait_timeout")
+qamw_calibrate_partial_sums = _raw("qamw_calibrate_partial_sums")
+qamw_sigma_from_partial_sums = _raw("qamw_sigma_from_partial_sums")
 qamw_lloyd_workspace_bytes = _raw("qamw_lloyd_workspace_bytes")
 qamw_lloyd_assign = _raw("qamw_lloyd_assign")
 qamw_lloyd_update = _raw("qamw_lloyd_update")
@@ -223,6 +228,55 @@ def calibrate_sigma(W, act_rms, alpha: float, block: int, seed: int, status=None
         _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
         _ptr(sigma), _ptr(workspace), workspace.numel(), _ptr(status), _stream_ptr(stream)))
     return sigma
+
+
+def calibrate_partial_sums(W, act_rms, alpha: float, block: int, seed: int, status=None, workspace=None,
+                           stream=None, out=None):
+    """fp64 [K/2] sums of |z_ik| over W's rows (one shard of a row-split matrix)."""
+    torch = _torch()
+    _need_cuda("W", W, ndim=2)
+    _need_cuda("act_rms", act_rms, torch.float32, 1)
+    M, K = W.shape
+    lib = load_library()
+    need = int(lib.qamw_calibrate_workspace_bytes(M, K))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    sums = torch.empty(K // 2, dtype=torch.float64, device=W.device) if out is None else out
+    _check("qamw_calibrate_partial_sums", lib.qamw_calibrate_partial_sums(
+        _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
+        _ptr(sums), _ptr(workspace), workspace.numel(), _ptr(status), _stream_ptr(stream)))
+    return sums
+
+
+def sigma_from_partial_sums(sums, M_total: int, stream=None, out=None):
+    """sigma [P] from the shards' sums (float64 [R][P], shard order)."""
+    torch = _torch()
+    _need_cuda("sums", sums, torch.float64, 2)
+    sums = sums.contiguous()
+    R, P = sums.shape
+    sigma = torch.empty(P, dtype=torch.float32, device=sums.device) if out is None else out
+    _check("qamw_sigma_from_partial_sums", load_library().qamw_sigma_from_partial_sums(
+        _ptr(sums), R, P, int(M_total), _ptr(sigma), _stream_ptr(stream)))
+    return sigma
+
+
+def gather_partial_sums(sums, group=None):
+    """All-gathers every rank's [P] sums into a [world, P] tensor in rank order
+    (one collective: NCCL over NVLink between GPUs, or gloo on CPU)."""
+    torch = _torch()
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    flat = torch.empty(world * sums.numel(), dtype=sums.dtype, device=sums.device)
+    dist.all_gather_into_tensor(flat, sums.contiguous().view(-1), group=group)
+    return flat.view(world, sums.numel())
+
+
+def calibrate_sigma_sharded(W_shard, act_rms, alpha: float, block: int, seed: int, M_total: int, group=None,
+                            status=None, stream=None):
+    """sigma of a matrix whose rows are split across the ranks of ``group``:
+    each rank passes its rows; every rank gets the same sigma."""
+    sums = calibrate_partial_sums(W_shard, act_rms, alpha, block, seed, status=status, stream=stream)
+    return sigma_from_partial_sums(gather_partial_sums(sums, group), M_total, stream=stream)
 
 
 @dataclass

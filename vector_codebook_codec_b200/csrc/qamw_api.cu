@@ -139,15 +139,15 @@ size_t qamw_calibrate_workspace_bytes(int64_t M, int64_t K) {
   return align256((size_t)K * 4) + align256((size_t)M * 4) + align256((size_t)groups * (size_t)(K / 2) * 8);
 }
 
-int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
-                         const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
-                         float *sigma_out, void *workspace, size_t workspace_bytes, int32_t *status,
-                         qamw_stream_t stream) {
-  static const char *fn = "qamw_calibrate_sigma";
-  CallRange nvtx_range(fn);
-  g_last_error[0] = 0;
+// Calibration of W's rows: sigma (sigma_out) or the fp64 sums of |z| per pair
+// position (sum_out) -- qamw_calibrate_sigma and qamw_calibrate_partial_sums.
+static int calibrate_impl(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                          const float *act_rms, float alpha, int32_t block, uint64_t sign_seed, float *sigma_out,
+                          double *sum_out, void *workspace, size_t workspace_bytes, int32_t *status,
+                          qamw_stream_t stream, const char *fn) {
   int rc;
-  if (W == nullptr || sigma_out == nullptr) return fail(QAMW_ENULL, "%s: W and sigma_out must be non-NULL", fn);
+  if (W == nullptr || (sigma_out == nullptr && sum_out == nullptr))
+    return fail(QAMW_ENULL, "%s: W and the output must be non-NULL", fn);
   if ((rc = check_dtype(w_dtype, fn))) return rc;
   if ((rc = check_shape(M, K, block, fn))) return rc;
   if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
@@ -171,8 +171,46 @@ int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K
   ca.partials = partials;
   ca.groups = (M + kCalibRowGroup - 1) / kCalibRowGroup;
   ca.sigma_out = sigma_out;
+  ca.sum_out = sum_out;
   if ((e = launch_calibrate(ca, st)) != cudaSuccess) return cuda_fail(e, fn);
   return QAMW_OK;
+}
+
+int qamw_calibrate_sigma(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                         const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                         float *sigma_out, void *workspace, size_t workspace_bytes, int32_t *status,
+                         qamw_stream_t stream) {
+  static const char *fn = "qamw_calibrate_sigma";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  if (sigma_out == nullptr) return fail(QAMW_ENULL, "%s: W and sigma_out must be non-NULL", fn);
+  return calibrate_impl(W, w_dtype, M, K, ldw, act_rms, alpha, block, sign_seed, sigma_out, nullptr, workspace,
+                        workspace_bytes, status, stream, fn);
+}
+
+int qamw_calibrate_partial_sums(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                                const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                                double *sums_out, void *workspace, size_t workspace_bytes, int32_t *status,
+                                qamw_stream_t stream) {
+  static const char *fn = "qamw_calibrate_partial_sums";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  if (sums_out == nullptr) return fail(QAMW_ENULL, "%s: W and sums_out must be non-NULL", fn);
+  return calibrate_impl(W, w_dtype, M, K, ldw, act_rms, alpha, block, sign_seed, nullptr, sums_out, workspace,
+                        workspace_bytes, status, stream, fn);
+}
+
+int qamw_sigma_from_partial_sums(const double *sums, int32_t R, int64_t P, int64_t M_total, float *sigma_out,
+                                 qamw_stream_t stream) {
+  static const char *fn = "qamw_sigma_from_partial_sums";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  if (!sums || !sigma_out) return fail(QAMW_ENULL, "%s: sums and sigma_out must be non-NULL", fn);
+  if (R < 1 || P < 1 || M_total < 1)
+    return fail(QAMW_EINVAL, "%s: R (%d), P (%lld) and M_total (%lld) must be >= 1", fn, R, (long long)P,
+                (long long)M_total);
+  cudaError_t e = launch_sigma_from_sums(sums, R, P, M_total, sigma_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
 }
 
 int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,

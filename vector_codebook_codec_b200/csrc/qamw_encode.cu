@@ -273,8 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate_kernel(CalibArgs a, int
 // g = w, w + 32, ... in order, then lane k of warp 0 adds the 32 warp sums in
 // order. The order depends only on the shape, never on the device.
 constexpr int kReduceWarps = 32;
+// With sum_out set, the kernel writes the fp64 sum instead of sigma (the
+// row-sharded calibration; see sigma_from_sums_kernel).
 __global__ void __launch_bounds__(kReduceWarps * 32) sigma_reduce_kernel(const double *partials, int64_t groups,
-                                                                         int64_t P, int64_t M, float *sigma_out) {
+                                                                         int64_t P, int64_t M, float *sigma_out,
+                                                                         double *sum_out) {
   __shared__ double part[kReduceWarps][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t k = (int64_t)blockIdx.x * 32 + lane;
@@ -287,11 +290,28 @@ __global__ void __launch_bounds__(kReduceWarps * 32) sigma_reduce_kernel(const d
     double t = 0.0;
 #pragma unroll
     for (int w = 0; w < kReduceWarps; ++w) t += part[w][lane];
-    const double c = 0.79788456080286535588;  // sqrt(2/pi)
-    float sg = (float)(c * (t / (double)M));
-    if (sg == 0.0f) sg = 1.0f;
-    sigma_out[k] = sg;
+    if (sum_out != nullptr) {
+      sum_out[k] = t;
+    } else {
+      const double c = 0.79788456080286535588;  // sqrt(2/pi)
+      float sg = (float)(c * (t / (double)M));
+      if (sg == 0.0f) sg = 1.0f;
+      sigma_out[k] = sg;
+    }
   }
+}
+
+// sigma_k from the sums of R row shards (rank order); R = 1 gives exactly the
+// value sigma_reduce_kernel writes for the whole matrix.
+__global__ void sigma_from_sums_kernel(const double *sums, int R, int64_t P, int64_t M, float *sigma_out) {
+  const int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (k >= P) return;
+  double t = 0.0;
+  for (int r = 0; r < R; ++r) t += sums[(int64_t)r * P + k];
+  const double c = 0.79788456080286535588;  // sqrt(2/pi)
+  float sg = (float)(c * (t / (double)M));
+  if (sg == 0.0f) sg = 1.0f;
+  sigma_out[k] = sg;
 }
 
 // ----------------------------------------------------------------------------
@@ -518,7 +538,13 @@ cudaError_t launch_calibrate(const CalibArgs &a, cudaStream_t s) {
   }
   const int64_t P = a.rot.K >> 1;
   sigma_reduce_kernel<<<(int)((P + 31) / 32), kReduceWarps * 32, 0, s>>>(a.partials, a.groups, P, a.rot.M,
-                                                                          a.sigma_out);
+                                                                          a.sigma_out, a.sum_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sigma_from_sums(const double *sums, int R, int64_t P, int64_t M, float *sigma_out,
+                                   cudaStream_t s) {
+  sigma_from_sums_kernel<<<(int)((P + 255) / 256), 256, 0, s>>>(sums, R, P, M, sigma_out);
   return cudaGetLastError();
 }
 

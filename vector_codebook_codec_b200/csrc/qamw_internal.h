@@ -65,6 +65,7 @@ struct CalibArgs {
   double *partials;      // [G][K/2]
   int64_t groups;        // G = ceil(M / kCalibRowGroup)
   float *sigma_out;      // [K/2]
+  double *sum_out = nullptr;  // [K/2]: if set, the fp64 sums are written instead of sigma
 };
 
 struct EncodeArgs {
@@ -112,6 +113,9 @@ struct RotateTestArgs {
 cudaError_t launch_channel_scale(const ScaleArgs &a, cudaStream_t s);
 cudaError_t launch_row_norms(const RowNormArgs &a, cudaStream_t s);
 cudaError_t launch_calibrate(const CalibArgs &a, cudaStream_t s);
+// sigma_k from R row shards' sums [R][P] added in rank order.
+cudaError_t launch_sigma_from_sums(const double *sums, int R, int64_t P, int64_t M, float *sigma_out,
+                                   cudaStream_t s);
 // The partial sums of the calibration for b <= 512 (qamw_calibrate.cu).
 cudaError_t launch_calibrate_partials512(const CalibArgs &a, cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
