@@ -186,7 +186,11 @@ int qamw_calibrate_sigma_noalloc(const void *W, qamw_dtype w_dtype, int64_t M, i
  *   codebook    : device float32 [N][2]
  *   search_table: device table from qamw_build_search_table for this codebook,
  *                 or NULL for the brute-force search over all N centroids.
- *                 Both searches return the same index.
+ *                 Both searches return the same index. The table is used for
+ *                 b <= 512 and N <= 2048; other shapes take the brute-force
+ *                 search (same result). A table that does not match the
+ *                 codebook (another N, a corrupt header) makes every pair
+ *                 scan all N centroids, still exact.
  *   packed_out  : device uint32 [M][qamw_words_per_row(K, bits)]
  *   row_norm_out: device float32 [M]                 col_scale_out: device float32 [K] (s_j)
  * row_norm_out and col_scale_out are the metadata qamw_decode needs; the

@@ -414,7 +414,7 @@ cudaError_t launch_tma_t(const DecodeArgs &a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   int warps = kMaxWarps;
   auto need = [&](int w, int copies) { return 1024 + (size_t)w * G::kWarpBytes + (size_t)a.N * copies * 8; };
-  // prefer 12 warps; shrink the table replication, then the warp count, to fit
+  // prefer kMaxWarps warps; shrink the table replication, then the warp count, to fit
   while (need(warps, ta.copies) > (size_t)smem_max && ta.copies > 4) ta.copies >>= 1;
   while (warps > 4 && need(warps, ta.copies) > (size_t)smem_max) --warps;
   while (need(warps, ta.copies) > (size_t)smem_max && ta.copies > 1) ta.copies >>= 1;
