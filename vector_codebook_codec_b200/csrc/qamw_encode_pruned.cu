@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ float s_a, s_UL, s_inv;
   if (threadIdx.x == 0) {
     const SearchHeader h = *reinterpret_cast<const SearchHeader *>(a.table);
-    const bool ok = h.magic == kSearchMagic && h.valid == 1 && h.N == N && h.G >= 1 && h.G <= 128 &&
+    const bool ok = h.magic == kSearchMagic && h.valid == 1 && h.N == N && h.G >= 1 && h.G <= 181 &&
                     h.G * h.G + 1 <= toff_slots && h.total >= 0 && h.total <= tab_cap - N &&
                     h.total + N < 65536 && h.a > 0.0f && h.UL > 0.0f && h.UL < 1.0f && h.inv_cw > 0.0f;
     s_use = ok ? 1 : 0;

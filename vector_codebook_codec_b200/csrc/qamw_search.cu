@@ -38,7 +38,9 @@
 
 namespace qamw {
 
-int search_grid(int N) { return N >= 64 ? 128 : 32; }
+// The finest grid whose table fits the encode's shared memory with 16-bit
+// offsets (lists + identity list < 65536 entries) for the shipped codebooks.
+int search_grid(int N) { return N >= 2048 ? 144 : (N >= 64 ? 160 : 32); }
 
 int64_t search_capacity(int N) {
   const int G = search_grid(N);
@@ -135,7 +137,7 @@ __global__ void table_count_kernel(const float *codebook, SearchHeader *h, uint3
 // threads, fixed order). Each thread owns up to kScanPer consecutive cells:
 // it keeps their counts in registers and writes only their offsets, so no
 // slot is read by one thread and written by another.
-constexpr int kScanPer = 16;   // 16384 cells (G = 128) / 1024 threads
+constexpr int kScanPer = 32;   // up to 32768 cells (G <= 181) / 1024 threads
 __global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint32_t *offsets) {
   __shared__ uint32_t wsum[32];
   const int n = h->G * h->G;
