@@ -198,9 +198,89 @@ def auto_rows(spec):
     return max(1, min(spec.M, int(round(64 * 2048 * 2048 / per_row))))
 
 
+def _reference_line(args, metric, value, unit, config, sample, ms_per_step, cores=1):
+    return {
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_reference_special(args):
+    """The oracle legs of the decode-only, polar and codebook-training workloads."""
+    import synth
+    import vector_codebook_codec_b200 as q
+    from oracle import codec
+    from oracle import lloyd as olloyd
+    if args.workload == "lloyd":
+        Ts = 1 << 18
+        x = synth.gaussian_points(LLOYD_T, LLOYD_SEED)[:Ts]
+        C = x[:LLOYD_N].copy()
+        idx = olloyd.assign(x, C)
+        for _ in range(args.warmup):
+            C = olloyd.centroid_update(x, idx, C)
+            idx = olloyd.assign(x, C)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            C = olloyd.centroid_update(x, idx, C)
+            idx = olloyd.assign(x, C)
+        dt = (time.perf_counter() - t0) / args.steps
+        value = (Ts / LLOYD_T) / dt
+        return _reference_line(args, "QAM-W codebook training: Lloyd iterations per second", value, "iterations/s",
+                               {"workload": "lloyd_N2048_T2097152", "N": LLOYD_N, "T": LLOYD_T},
+                               f"{Ts} of {LLOYD_T} samples per iteration, scaled", 1e3 / value, os.cpu_count())
+    if args.workload == "polar":
+        spec = synth.llama7b_attn().specs[0]
+        _, W32 = synth.to_bf16(synth.make_matrix(spec))
+        act = synth.act_for(spec)
+        pol = q.load_polar(spec.N)
+        rows = args.cpu_rows or 64
+        sig = codec.calibrate_sigma(W32[:rows], act, spec.alpha, spec.block, spec.seed)
+        ts = []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            e = codec.encode_polar(W32[:rows], act, spec.alpha, spec.block, spec.seed, sig, pol["amps"], pol["P"],
+                                   spec.bits)
+            codec.decode_with_scale(e["idx"], e["r"], sig, e["s"], spec.K, spec.block, spec.seed, pol["points"])
+            if i >= args.warmup:
+                ts.append(time.perf_counter() - t0)
+        value = rows * spec.K * len(ts) / sum(ts) / 1e9
+        return _reference_line(args, METRIC, value, "Gweights/s",
+                               {"workload": "polar_4096x4096_bf16_b128_A32xP64", "codec": "polar baseline"},
+                               f"{rows} of {spec.M} rows per step (polar encode + decode)", 1e3 * sum(ts) / len(ts))
+    # decode_13b: decode only, on row samples of the three matrices
+    wl = synth.decode_sweep_13b()
+    rows = args.cpu_rows or 16
+    ts, weights = [], 0
+    for i in range(args.warmup + args.steps):
+        t = 0.0
+        for spec in wl.specs:
+            idx = synth.make_indices(rows, spec.K // 2, spec.N, spec.seed)
+            r = synth.make_row_norms(rows, spec.seed)
+            sig = synth.make_sigma(spec.K // 2, spec.seed)
+            s_ = synth.make_act_rms(spec.K, 0.5, spec.seed)
+            C = q.load_codebook(spec.N)
+            t0 = time.perf_counter()
+            codec.decode_with_scale(idx, r, sig, s_, spec.K, spec.block, spec.seed, C)
+            t += time.perf_counter() - t0
+            if i == 0:
+                weights += rows * spec.K
+        if i >= args.warmup:
+            ts.append(t)
+    value = weights * len(ts) / sum(ts) / 1e9
+    return _reference_line(args, METRIC, value, "Gweights/s",
+                           {"workload": wl.name, "op": "decode only"},
+                           f"{rows} rows of each 13B-shaped matrix per step (decode)", 1e3 * sum(ts) / len(ts))
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
+        return 0
+    if args.workload in ("lloyd", "polar", "decode_13b"):
+        print(json.dumps(run_reference_special(args)), flush=True)
         return 0
     import synth
     import vector_codebook_codec_b200 as q
