@@ -7,6 +7,8 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -82,6 +84,25 @@ int g_sm_count[64] = {0};
 }  // namespace
 
 void set_last_error(const char *msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
+cudaError_t set_max_dynamic_smem(const void *func, size_t bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<const void *, int>, size_t>> done;   // (kernel, device) -> bytes set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto &d : done)
+    if (d.first.first == func && d.first.second == dev) {
+      if (d.second >= bytes) return cudaSuccess;
+      if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) == cudaSuccess)
+        d.second = bytes;
+      return e;
+    }
+  if ((e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) == cudaSuccess)
+    done.push_back({{func, dev}, bytes});
+  return e;
+}
 
 int sm_count() {
   int dev = 0;

@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate512_kernel(CalibArgs a, 
 
 template <typename Kern>
 cudaError_t set_smem(Kern k, size_t bytes) {
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return set_max_dynamic_smem(reinterpret_cast<const void *>(k), bytes);
 }
 
 template <int WT>

@@ -484,7 +484,7 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
   while (warps > 1 && cb_bytes + (size_t)warps * g.warp_bytes > (size_t)smem_max) --warps;
   const size_t smem = cb_bytes + (size_t)warps * g.warp_bytes;
   if (smem > (size_t)smem_max) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(decode_kernel<BITS, LB, BF16OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = set_max_dynamic_smem(reinterpret_cast<const void *>(decode_kernel<BITS, LB, BF16OUT>), smem);
   if (e != cudaSuccess) return e;
   const int fast_store = (reinterpret_cast<uintptr_t>(a.out) % 16 == 0) && ((a.ldo * kEs) % 16 == 0);
   const int vec_words = (reinterpret_cast<uintptr_t>(a.packed) % 8 == 0) && (a.wpr % 2 == 0);

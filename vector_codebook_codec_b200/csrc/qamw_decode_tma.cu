@@ -425,7 +425,7 @@ cudaError_t launch_tma_t(const DecodeArgs &a, cudaStream_t s) {
   ta.n_bands = (a.M + G::kRows - 1) / G::kRows;
   ta.n_tasks = ta.n_segcols * ta.n_bands;
   const size_t smem = need(warps, ta.copies);
-  e = cudaFuncSetAttribute(decode_tma_kernel<BITS, LB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = set_max_dynamic_smem(reinterpret_cast<const void *>(decode_tma_kernel<BITS, LB>), smem);
   if (e != cudaSuccess) return e;
   // one CTA per SM; every column strip needs at least one warp
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((ta.n_tasks + warps - 1) / warps, sm_count()));

@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kThreads) rotate_test_kernel(RotateTestArgs a)
 
 template <typename Kern>
 cudaError_t set_smem(Kern k, size_t bytes) {
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return set_max_dynamic_smem(reinterpret_cast<const void *>(k), bytes);
 }
 
 bool w_vec_ok(const void *W, qamw_dtype wt, int64_t ldw) {

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) encode_polar_kernel(EncodeArg
 template <int WT>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
   const size_t smem = kUnitSmemBytes + (size_t)std::max(a.polar_A - 1, 1) * sizeof(double);
-  cudaError_t e = cudaFuncSetAttribute(encode_polar_kernel<WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(encode_polar_kernel<WT>), smem);
   if (e != cudaSuccess) return e;
   const int64_t n_chunks = (a.rot.K + kUnit - 1) / kUnit;
   const int64_t tiles = n_chunks * ((a.rot.M + kUnitWarps - 1) / kUnitWarps);

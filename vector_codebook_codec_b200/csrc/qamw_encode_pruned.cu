@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <typename Kern>
 cudaError_t set_smem(Kern k, size_t bytes) {
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return set_max_dynamic_smem(reinterpret_cast<const void *>(k), bytes);
 }
 
 template <int WT>

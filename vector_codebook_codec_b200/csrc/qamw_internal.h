@@ -144,6 +144,11 @@ cudaError_t launch_lloyd_update(const double *pts, int64_t T, const int32_t *idx
 // Test hook: a bounded wait on an mbarrier that never completes (qamw_selftest.cu).
 cudaError_t launch_wait_timeout(uint32_t tries, int32_t *status, cudaStream_t s);
 
+// cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) on the current
+// device, once per (kernel, device) and size: later calls with a size already
+// set cost a lookup instead of a driver call.
+cudaError_t set_max_dynamic_smem(const void *func, size_t bytes);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

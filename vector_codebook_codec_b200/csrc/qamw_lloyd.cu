@@ -145,7 +145,7 @@ size_t lloyd_workspace_bytes(int64_t T, int N) {
 cudaError_t launch_lloyd_assign(const double *pts, int64_t T, const double *cent, int N, int32_t *idx,
                                 unsigned long long *changed, cudaStream_t s) {
   const size_t smem = (size_t)N * sizeof(double2);
-  cudaError_t e = cudaFuncSetAttribute(lloyd_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(lloyd_assign_kernel), smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((T + kAssignThreads - 1) / kAssignThreads,
                                                                 (int64_t)sm_count() * 8));
