@@ -1,10 +1,10 @@
 #!/usr/bin/env python
 """QAM-W codec benchmark: encode/decode Gweights/s of one weight matrix per step.
 
-A *step* is one pass of the whole hot path over one matrix: qamw_calibrate_sigma
-(sigma_k), qamw_encode (channel scale, row norms, rotation, nearest-centroid
-search, packing) and qamw_decode (bf16 weights), all through the C ABI of
-libqamw.so. The default workload is the Llama-7B-shaped attention projection:
+A *step* is one pass of the whole hot path over one matrix:
+qamw_calibrate_encode (channel scale and row norms once, then the sigma_k
+calibration pass and the encode pass: rotation, nearest-centroid search,
+packing) and qamw_decode (bf16 weights), all through the C ABI of libqamw.so. The default workload is the Llama-7B-shaped attention projection:
 bf16 4096 x 4096, N(0, 0.02^2) with 0.5% outlier columns x20, act RMS
 lognormal(0, 1), alpha 0.5, Hadamard block 128, 2048 centroids (11 bits per
 pair). Inputs are synthetic (seeded); the codebook is the shipped Lloyd table.
@@ -723,18 +723,29 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(max(args.steps, 1))]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(max(args.steps, 1))]
+    bd = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(max(args.steps, 1))]
 
     def one(evs=None):
+        """The step: calibrate + encode in one call (s and r computed once), then decode."""
         if evs: evs[0].record(stream)
+        enc = q.calibrate_encode(Wd, actd, spec.alpha, spec.block, spec.seed, Cd, spec.bits, status=status,
+                                 out=(packed, rnorm, cscale, sigma), search_table=table, workspace=ws)
+        if evs: evs[1].record(stream)
+        q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=out)
+        if evs: evs[2].record(stream)
+
+    def separate(evs):
+        """The same work as three separate calls, for the per-call breakdown."""
+        evs[0].record(stream)
         sig = q.calibrate_sigma(Wd, actd, spec.alpha, spec.block, spec.seed, status=status, workspace=ws,
                                 out=sigma)
-        if evs: evs[1].record(stream)
+        evs[1].record(stream)
         enc = q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sig, Cd, spec.bits, status=status,
                        out=(packed, rnorm, cscale), search_table=table)
-        if evs: evs[2].record(stream)
+        evs[2].record(stream)
         q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=out)
-        if evs: evs[3].record(stream)
+        evs[3].record(stream)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -743,20 +754,19 @@ def run_ours(args):
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()} after warm-up")
 
-    # The same step captured once as a CUDA graph (its 8 kernels replayed as one
+    # The same step captured once as a CUDA graph (its 6 kernels replayed as one
     # graph launch: the launch gaps between dependent kernels shrink). The
-    # headline is the replayed step; the eager calls below give the per-call
-    # breakdown. Both run the same kernels on the same buffers.
+    # headline is the replayed step; the eager calls below time it call by
+    # call. Both run the same kernels on the same buffers.
     graph = None
     if args.graph:
         side = torch.cuda.Stream(dev)
         graph = torch.cuda.CUDAGraph()
         torch.cuda.synchronize(dev)
         with torch.cuda.graph(graph, stream=side):
-            q.calibrate_sigma(Wd, actd, spec.alpha, spec.block, spec.seed, status=status, workspace=ws, out=sigma,
-                              stream=side)
-            genc = q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sigma, Cd, spec.bits, status=status,
-                            out=(packed, rnorm, cscale), search_table=table, stream=side)
+            genc = q.calibrate_encode(Wd, actd, spec.alpha, spec.block, spec.seed, Cd, spec.bits, status=status,
+                                      out=(packed, rnorm, cscale, sigma), search_table=table, workspace=ws,
+                                      stream=side)
             q.decode(genc, Cd, out_dtype=torch.bfloat16, status=status, out=out, stream=side)
         for _ in range(args.warmup):
             flush.fill_(3.0)
@@ -775,6 +785,10 @@ def run_ours(args):
         flush.fill_(float(i))
         one(ev[i])
     torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(float(i) + 0.25)
+        separate(bd[i])
+    torch.cuda.synchronize(dev)
     if graph is not None:
         if world > 1:
             dist.barrier()
@@ -791,10 +805,11 @@ def run_ours(args):
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()} in the timed steps")
 
-    t_cal = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    t_enc = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    t_dec = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
-    t_step = [ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    t_cal = [bd[i][0].elapsed_time(bd[i][1]) for i in range(args.steps)]
+    t_enc = [bd[i][1].elapsed_time(bd[i][2]) for i in range(args.steps)]
+    t_dec = [bd[i][2].elapsed_time(bd[i][3]) for i in range(args.steps)]
+    t_calenc = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    t_step = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
     total_s = max_over_ranks(sum(t_step) / 1e3, dev)      # eager steps
     weights = M * K
     value = aggregate_throughput(weights * args.steps, total_s, world) / 1e9
@@ -901,11 +916,9 @@ def run_ours(args):
             with torch.cuda.stream(s_comp):
                 s_comp.wait_event(sl["h2d"])
                 s_comp.wait_event(sl["d2h"])            # step i-2's results have been read back
-                sg = q.calibrate_sigma(sl["W"], sl["act"], spec.alpha, spec.block, spec.seed, status=status,
-                                       workspace=sl["ws"], out=sl["sigma"], stream=s_comp)
-                enc = q.encode(sl["W"], sl["act"], spec.alpha, spec.block, spec.seed, sg, Cd, spec.bits,
-                               status=status, out=(sl["packed"], sl["r"], sl["s"]), search_table=table,
-                               stream=s_comp)
+                enc = q.calibrate_encode(sl["W"], sl["act"], spec.alpha, spec.block, spec.seed, Cd, spec.bits,
+                                         status=status, out=(sl["packed"], sl["r"], sl["s"], sl["sigma"]),
+                                         search_table=table, workspace=sl["ws"], stream=s_comp)
                 q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=sl["out"], stream=s_comp)
                 sl["comp"].record(s_comp)
             with torch.cuda.stream(s_d2h):
@@ -965,10 +978,13 @@ def run_ours(args):
                        "parallelism": f"{world} independent replica(s)"},
             "roofline": enc_roof,
             "rooflines": rooflines,
-            "ms": {"calibrate": cal_ms, "encode": enc_ms, "decode": dec_ms},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 8 * args.steps, "clocks": clk,
-            "timing": ("each step replays a CUDA graph of the 8 kernels (captured once from the C-ABI calls); "
-                       "'eager' and 'ms' are the same step launched call by call" if args.graph else
+            "ms": {"calibrate": cal_ms, "encode": enc_ms, "decode": dec_ms,
+                   "calibrate_encode": statistics.mean(t_calenc),
+                   "note": ("calibrate, encode and decode: the three separate calls (each computes s and r); "
+                            "calibrate_encode: the step's fused call (s and r once)")},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 6 * args.steps, "clocks": clk,
+            "timing": ("each step replays a CUDA graph of the 6 kernels (captured once from the C-ABI calls); "
+                       "'eager' is the same step launched call by call" if args.graph else
                        "each step launched call by call"),
             "eager": eager,
             "dtype_detail": "rotation fp64, search and decode fp32, decode output bf16",

@@ -204,6 +204,29 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
                 float *col_scale_out, int32_t *status, qamw_stream_t stream);
 
 /*
+ * qamw_calibrate_encode -- qamw_calibrate_sigma followed by qamw_encode on the
+ * same matrix, as one call: Methodology (3) calibrates sigma over the rows of
+ * W, then steps (5), (1), (2), (3), (4) code them with that sigma. The channel
+ * scales s_j (step 5) and the row norms r_i (step 1) are computed once, into
+ * col_scale_out and row_norm_out, and read by both passes; the two separate
+ * calls compute each of them twice. Every output equals, bit for bit, what
+ * qamw_calibrate_sigma and then qamw_encode (with sigma_out as its sigma)
+ * write.
+ * (An interface of this library; the QAM-W page has no counterpart.)
+ *   sigma_out : device float32 [K/2]   workspace: device, 256-byte aligned,
+ *               >= qamw_calibrate_workspace_bytes(M, K)
+ *   other arguments as qamw_encode; packed_out, row_norm_out and
+ *   col_scale_out are qamw_encode's outputs, and the calibration reads
+ *   row_norm_out and col_scale_out after writing them.
+ * Errors: as qamw_encode, plus QAMW_EWORKSPACE.
+ */
+int qamw_calibrate_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                          const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                          const float *codebook, int32_t N, int32_t bits_per_pair, const void *search_table,
+                          float *sigma_out, uint32_t *packed_out, float *row_norm_out, float *col_scale_out,
+                          void *workspace, size_t workspace_bytes, int32_t *status, qamw_stream_t stream);
+
+/*
  * qamw_search_table_bytes / qamw_build_search_table -- an exact pruned search
  * for Methodology (4): a grid over the plane of normalised pairs, each cell
  * listing (in ascending index order) every centroid that can be the fp32

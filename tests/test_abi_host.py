@@ -124,6 +124,31 @@ def test_calibrate_rejects_on_host(lib, kw, code):
     assert _cal(lib, **kw) == code
 
 
+def _cal_enc(lib, **kw):
+    a = dict(W=FAKE, wt=1, M=8, K=256, ldw=256, act=None, alpha=0.5, block=128, seed=1, cb=FAKE, N=256,
+             bits=8, table=None, sigma=FAKE, packed=FAKE, r=FAKE, s=FAKE, ws=FAKE, wsb=1 << 30, status=None,
+             stream=None)
+    a.update(kw)
+    return lib.qamw_calibrate_encode(a["W"], a["wt"], a["M"], a["K"], a["ldw"], a["act"], a["alpha"],
+                                     a["block"], a["seed"], a["cb"], a["N"], a["bits"], a["table"], a["sigma"],
+                                     a["packed"], a["r"], a["s"], a["ws"], a["wsb"], a["status"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(W=None), QAMW_ENULL), (dict(cb=None), QAMW_ENULL), (dict(sigma=None), QAMW_ENULL),
+    (dict(packed=None), QAMW_ENULL), (dict(r=None), QAMW_ENULL), (dict(s=None), QAMW_ENULL),
+    (dict(ws=None), QAMW_EWORKSPACE), (dict(wsb=16), QAMW_EWORKSPACE),
+    (dict(ws=ctypes.c_void_p(0x10010)), QAMW_EINVAL), (dict(K=255, ldw=255), QAMW_EINVAL),
+    (dict(block=96), QAMW_EINVAL), (dict(M=0), QAMW_EINVAL), (dict(ldw=128), QAMW_EINVAL),
+    (dict(N=257), QAMW_EINVAL), (dict(bits=17), QAMW_EINVAL), (dict(alpha=float("nan")), QAMW_EINVAL),
+    (dict(wt=7), QAMW_EINVAL), (dict(table=ctypes.c_void_p(0x10008)), QAMW_EINVAL),
+    (dict(block=2048, K=2048, ldw=2048), QAMW_EUNSUPPORTED),
+])
+def test_calibrate_encode_rejects_on_host(lib, kw, code):
+    assert _cal_enc(lib, **kw) == code
+    assert lib.qamw_last_error()
+
+
 def test_rotate_and_scale_reject_on_host(lib):
     assert lib.qamw_rotate_rows(None, FAKE, 2, 8, 4, 0, 0, None) == QAMW_ENULL
     assert lib.qamw_rotate_rows(FAKE, FAKE, 2, 12, 8, 0, 0, None) == QAMW_EINVAL

@@ -47,6 +47,9 @@ _SIGNATURES = {
                                             _c_u64, _c_p, _c_p, _c_sz, _c_p, _c_p]),
     "qamw_encode": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32, _c_u64,
                                    _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
+    "qamw_calibrate_encode": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32, _c_i32,
+                                             _c_u64, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                             _c_sz, _c_p, _c_p]),
     "qamw_decode": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
                                    _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
@@ -117,6 +120,7 @@ qamw_channel_scale = _raw("qamw_channel_scale")
 qamw_calibrate_workspace_bytes = _raw("qamw_calibrate_workspace_bytes")
 qamw_calibrate_sigma = _raw("qamw_calibrate_sigma")
 qamw_encode = _raw("qamw_encode")
+qamw_calibrate_encode = _raw("qamw_calibrate_encode")
 qamw_decode = _raw("qamw_decode")
 qamw_rotate_rows = _raw("qamw_rotate_rows")
 qamw_encode_polar = _raw("qamw_encode_polar")
@@ -335,6 +339,38 @@ def encode(W, act_rms, alpha: float, block: int, seed: int, sigma, codebook, bit
         _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
         _ptr(sigma), _ptr(codebook.contiguous()), N, bits, _ptr(search_table), _ptr(packed), _ptr(r), _ptr(s),
         _ptr(status), _stream_ptr(stream)))
+    return Encoded(packed, r, s, sigma, M, K, block, seed, N, bits)
+
+
+def calibrate_encode(W, act_rms, alpha: float, block: int, seed: int, codebook, bits: int,
+                     status=None, stream=None, out=None, search_table=None, workspace=None) -> Encoded:
+    """:func:`calibrate_sigma` then :func:`encode` in one call (qamw_calibrate_encode):
+    s_j and r_i are computed once; the result equals the two calls' bit for bit.
+    ``out`` = (packed, row_norm, col_scale, sigma) preallocated, or None."""
+    torch = _torch()
+    _need_cuda("W", W, ndim=2)
+    _need_cuda("act_rms", act_rms, torch.float32, 1)
+    _need_cuda("codebook", codebook, torch.float32, 2)
+    M, K = W.shape
+    N = codebook.shape[0]
+    wpr = words_per_row(K, bits)
+    if wpr < 0:
+        raise ValueError("invalid K / bits")
+    lib = load_library()
+    need = int(lib.qamw_calibrate_workspace_bytes(M, K))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    if out is None:
+        packed = torch.empty((M, wpr), dtype=torch.int32, device=W.device)
+        r = torch.empty(M, dtype=torch.float32, device=W.device)
+        s = torch.empty(K, dtype=torch.float32, device=W.device)
+        sigma = torch.empty(K // 2, dtype=torch.float32, device=W.device)
+    else:
+        packed, r, s, sigma = out
+    _check("qamw_calibrate_encode", lib.qamw_calibrate_encode(
+        _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(act_rms), float(alpha), block, seed & (2**64 - 1),
+        _ptr(codebook.contiguous()), N, bits, _ptr(search_table), _ptr(sigma), _ptr(packed), _ptr(r), _ptr(s),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream_ptr(stream)))
     return Encoded(packed, r, s, sigma, M, K, block, seed, N, bits)
 
 

@@ -273,6 +273,63 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
   return QAMW_OK;
 }
 
+int qamw_calibrate_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                          const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
+                          const float *codebook, int32_t N, int32_t bits_per_pair, const void *search_table,
+                          float *sigma_out, uint32_t *packed_out, float *row_norm_out, float *col_scale_out,
+                          void *workspace, size_t workspace_bytes, int32_t *status, qamw_stream_t stream) {
+  static const char *fn = "qamw_calibrate_encode";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  int rc;
+  if (!W || !codebook || !sigma_out || !packed_out || !row_norm_out || !col_scale_out)
+    return fail(QAMW_ENULL,
+                "%s: W, codebook, sigma_out, packed_out, row_norm_out, col_scale_out must be non-NULL", fn);
+  if ((rc = check_dtype(w_dtype, fn))) return rc;
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if ((rc = check_code(N, bits_per_pair, fn))) return rc;
+  if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
+  if (!std::isfinite(alpha)) return fail(QAMW_EINVAL, "%s: alpha must be finite", fn);
+  if (search_table != nullptr && reinterpret_cast<uintptr_t>(search_table) % 16)
+    return fail(QAMW_EINVAL, "%s: search_table must be 16-byte aligned", fn);
+  const size_t need = qamw_calibrate_workspace_bytes(M, K);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(QAMW_EWORKSPACE, "%s: workspace of %zu bytes needed (got %zu)", fn, need, workspace_bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(QAMW_EINVAL, "%s: workspace must be 256-byte aligned", fn);
+  // the partials sit where qamw_calibrate_sigma puts them; s and r go straight
+  // to the caller's metadata arrays, which both passes read
+  double *partials = reinterpret_cast<double *>(static_cast<unsigned char *>(workspace) + align256((size_t)K * 4) +
+                                                align256((size_t)M * 4));
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = launch_channel_scale(ScaleArgs{act_rms, alpha, K, col_scale_out, status}, st)) != cudaSuccess)
+    return cuda_fail(e, fn);
+  if ((e = launch_row_norms(RowNormArgs{W, w_dtype, M, K, ldw, col_scale_out, row_norm_out, status}, st)) !=
+      cudaSuccess)
+    return cuda_fail(e, fn);
+  const RotateArgs rot{W, w_dtype, M, K, ldw, log2i(block), sign_seed, col_scale_out, row_norm_out};
+  CalibArgs ca;
+  ca.rot = rot;
+  ca.partials = partials;
+  ca.groups = (M + kCalibRowGroup - 1) / kCalibRowGroup;
+  ca.sigma_out = sigma_out;
+  ca.sum_out = nullptr;
+  if ((e = launch_calibrate(ca, st)) != cudaSuccess) return cuda_fail(e, fn);
+  EncodeArgs ea;
+  ea.rot = rot;
+  ea.sigma = sigma_out;
+  ea.codebook = codebook;
+  ea.N = N;
+  ea.bits = bits_per_pair;
+  ea.wpr = qamw_words_per_row(K, bits_per_pair);
+  ea.packed = packed_out;
+  ea.table = search_table;
+  ea.status = status;
+  if ((e = launch_encode(ea, st)) != cudaSuccess) return cuda_fail(e, fn);
+  return QAMW_OK;
+}
+
 int qamw_encode_polar(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
                       const float *act_rms, float alpha, int32_t block, uint64_t sign_seed, const float *sigma,
                       const double *amps, int32_t A, int32_t P, int32_t bits_per_pair, uint32_t *packed_out,
