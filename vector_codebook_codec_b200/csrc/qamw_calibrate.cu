@@ -41,8 +41,8 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate512_kernel(CalibArgs a, 
   const int64_t t0 = (int64_t)blockIdx.x * T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
   const double inv_sqrt_b = 1.0 / sqrt((double)(1 << ra.log2b));
 
-  auto prefetch = [&](int64_t t, WRegs<WT> &w, float &rn) -> bool {
-    const int64_t chunk = t / RG, row = (t % RG) * kTileRows + warp;
+  auto prefetch = [&](int64_t chunk, int64_t g, WRegs<WT> &w, float &rn) -> bool {
+    const int64_t row = g * kTileRows + warp;
     rn = 0.0f;
     if (row >= M) return false;
     rn = ra.r[row];
@@ -51,11 +51,15 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate512_kernel(CalibArgs a, 
 
   WRegs<WT> wn;
   float rn_next = 0.0f;
-  bool full_next = (t0 < t1) ? prefetch(t0, wn, rn_next) : false;
+  // tile t = chunk * RG + g, walked incrementally (no 64-bit division per tile)
+  int64_t chunk = t0 / RG, g = t0 % RG, next_chunk = chunk, next_g = g;
+  bool full_next = (t0 < t1) ? prefetch(chunk, g, wn, rn_next) : false;
   int64_t cur_chunk = -1;
   int buf = 0;
-  for (int64_t t = t0; t < t1; ++t, buf ^= 1) {
-    const int64_t chunk = t / RG, g = t % RG;
+  for (int64_t t = t0; t < t1; ++t, buf ^= 1, chunk = next_chunk, g = next_g) {
+    next_g = g + 1;
+    next_chunk = chunk;
+    if (next_g == RG) { next_g = 0; ++next_chunk; }
     if (chunk != cur_chunk) {
       __syncthreads();
       if (threadIdx.x < kUnit) load_sd512(sm.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
@@ -65,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 1) calibrate512_kernel(CalibArgs a, 
     const WRegs<WT> wc = wn;
     const bool full = full_next;
     const float r = rn_next;
-    if (t + 1 < t1) full_next = prefetch(t + 1, wn, rn_next);
+    if (t + 1 < t1) full_next = prefetch(next_chunk, next_g, wn, rn_next);
 
     const int64_t row = g * kTileRows + warp;
     double acc[8];

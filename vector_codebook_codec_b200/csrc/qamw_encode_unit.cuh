@@ -59,8 +59,8 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
   const uint64_t divB = (0x100000000ull / (uint64_t)B) + 1ull;
 
   // the next unit's weights and row norm, loaded while the current one is searched
-  auto prefetch = [&](int64_t t, WRegs<WT> &w, float &rn) -> bool {
-    const int64_t chunk = t / RG, row = (t % RG) * kUnitWarps + warp;
+  auto prefetch = [&](int64_t chunk, int64_t g, WRegs<WT> &w, float &rn) -> bool {
+    const int64_t row = g * kUnitWarps + warp;
     rn = 0.0f;
     if (row >= M) return false;
     rn = ra.r[row];
@@ -69,10 +69,14 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
 
   WRegs<WT> wn;
   float rn_next = 0.0f;
-  bool full_next = (t0 < t1) ? prefetch(t0, wn, rn_next) : false;
+  // tile t = chunk * RG + g, walked incrementally (no 64-bit division per tile)
+  int64_t chunk = t0 / RG, g = t0 % RG, next_chunk = chunk, next_g = g;
+  bool full_next = (t0 < t1) ? prefetch(chunk, g, wn, rn_next) : false;
   int64_t cur_chunk = -1;
-  for (int64_t t = t0; t < t1; ++t) {
-    const int64_t chunk = t / RG, g = t % RG;
+  for (int64_t t = t0; t < t1; ++t, chunk = next_chunk, g = next_g) {
+    next_g = g + 1;
+    next_chunk = chunk;
+    if (next_g == RG) { next_g = 0; ++next_chunk; }
     if (chunk != cur_chunk) {
       __syncthreads();   // every warp is done with the previous chunk's tables (and the table copy is complete)
       if (threadIdx.x < kUnit) load_sd512(ct.sd, ra.s, ra.seed, K, chunk, threadIdx.x);
@@ -92,7 +96,7 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
     const WRegs<WT> wc = wn;
     const bool full = full_next;
     const float r = rn_next;
-    if (t + 1 < t1) full_next = prefetch(t + 1, wn, rn_next);
+    if (t + 1 < t1) full_next = prefetch(next_chunk, next_g, wn, rn_next);
 
     const int64_t row = g * kUnitWarps + warp;
     if (row >= M) continue;

@@ -15,10 +15,24 @@
 // For a pair x in Q its exact nearest distance d* is at most D(Q), and every
 // centroid whose fp32 direct-difference distance ties or beats the fp32
 // distance of the exact nearest one is within a factor (1 + 4e-7) of d*, so
-// it is listed. Scanning a cell's list in ascending index order with a strict
-// "<" therefore returns exactly the index of the brute-force search (the
-// lowest index among the fp32 minimisers). Pairs outside the grid, or a table
-// that does not fit, use the brute-force search.
+// it passes this first test.
+//
+// The first test keeps every centroid whose disc of radius D(Q) meets Q; a
+// second one drops the members that another member beats everywhere in Q.
+// Member c is dropped if some member c' has
+//     |p - c|^2 > (1 + 1e-5) |p - c'|^2   at the four corners p of Q.
+// f(p) = |p - c|^2 - (1 + 1e-5) |p - c'|^2 is -1e-5 |p|^2 plus terms of degree
+// at most one, a concave function, so its least value over the rectangle Q is
+// taken at a corner: f > 0 at the corners means f > 0 on all of Q. The fp32
+// distances of c and c' are within a factor (1 + 4e-7) of the exact ones, so
+// at every pair in Q the fp32 distance of c is strictly greater than that of
+// c': c is never the fp32 minimiser nor tied with it. (If c' is dropped in
+// turn, the member that beats c' beats c too.) The fp32 minimisers of every
+// pair in Q are therefore all kept, and scanning a cell's list in ascending
+// index order with a strict "<" returns exactly the index of the brute-force
+// search (the lowest index among the fp32 minimisers). A first-test list longer
+// than kListMax is kept whole. Pairs outside the grid, or a table that does
+// not fit, use the brute-force search.
 //
 // The encode computes a pair's cell in fp32 as floor((T(x) + UL) * inv_cw)
 // with UL, inv_cw and a read from the header; its rounding error is below
@@ -40,7 +54,7 @@ namespace qamw {
 
 // The finest grid whose table fits the encode's shared memory with 16-bit
 // offsets (lists + identity list < 65536 entries) for the shipped codebooks.
-int search_grid(int N) { return N >= 2048 ? 144 : (N >= 64 ? 160 : 32); }
+int search_grid(int N) { return N >= 2048 ? 176 : (N >= 64 ? 160 : 32); }
 
 int64_t search_capacity(int N) {
   const int G = search_grid(N);
@@ -58,6 +72,8 @@ namespace {
 constexpr double kCellMargin = 1e-3;   // cell enlargement, in cells (covers fp32 rounding of the cell index)
 constexpr double kTieSlack = 1e-5;     // relative slack on D(Q)^2
 constexpr float kAxisA = 2.0f;         // T(x) = x / (a + |x|): cells about 1/4 as wide at 0 as near |x| = 2
+constexpr int kListMax = 256;          // first-test members a warp prunes (shared-memory buffer per warp)
+constexpr int kListThreads = 256;      // threads per CTA of the count and fill kernels (one warp per cell)
 
 __global__ void table_header_kernel(const float *codebook, int N, int G, int64_t capacity, SearchHeader *h) {
   __shared__ float red[32];
@@ -119,17 +135,66 @@ __device__ double cell_bound(const float *codebook, int N, double x0, double x1,
   return d * (1.0 + kTieSlack);
 }
 
-__global__ void table_count_kernel(const float *codebook, SearchHeader *h, uint32_t *offsets) {
+// The members of the cell's first-test list, ascending, into the warp's buffer
+// (when there are at most kListMax of them); returns their number.
+__device__ int first_test(const float *codebook, int N, double x0, double x1, double y0, double y1, int lane,
+                          uint16_t *buf) {
+  const double bound = cell_bound(codebook, N, x0, x1, y0, y1, lane);
+  int n = 0;
+  for (int base = 0; base < N; base += 32) {
+    const int i = base + lane;
+    const bool in = i < N && dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
+    const uint32_t m = __ballot_sync(0xffffffffu, in);
+    const int at = n + __popc(m & ((1u << lane) - 1u));
+    if (in && at < kListMax) buf[at] = (uint16_t)i;
+    n += __popc(m);
+  }
+  __syncwarp();
+  return n;
+}
+
+// Whether member k of the buffer is beaten at all four corners of the cell by
+// another member (the second test).
+__device__ bool beaten(const float *codebook, const uint16_t *buf, int n, int k, double x0, double x1, double y0,
+                       double y1) {
+  const double px[4] = {x0, x0, x1, x1}, py[4] = {y0, y1, y0, y1};
+  const int c = buf[k];
+  const double cx = codebook[2 * c], cy = codebook[2 * c + 1];
+  double dc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dc[q] = (px[q] - cx) * (px[q] - cx) + (py[q] - cy) * (py[q] - cy);
+  for (int j = 0; j < n; ++j) {
+    if (j == k) continue;
+    const int o = buf[j];
+    const double ox = codebook[2 * o], oy = codebook[2 * o + 1];
+    bool all = true;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const double d = (px[q] - ox) * (px[q] - ox) + (py[q] - oy) * (py[q] - oy);
+      all = all && (dc[q] > (1.0 + kTieSlack) * d);
+    }
+    if (all) return true;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(kListThreads) table_count_kernel(const float *codebook, SearchHeader *h,
+                                                                   uint32_t *offsets) {
+  __shared__ uint16_t bufs[kListThreads / 32][kListMax];
   const int lane = threadIdx.x & 31;
+  uint16_t *buf = bufs[threadIdx.x >> 5];
   const int cell = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
   const SearchHeader hh = *h;
   if (cell >= hh.G * hh.G) return;
   double x0, x1, y0, y1;
   cell_bounds(hh, cell, x0, x1, y0, y1);
-  const double bound = cell_bound(codebook, hh.N, x0, x1, y0, y1, lane);
-  int cnt = 0;
-  for (int i = lane; i < hh.N; i += 32) cnt += dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  const int n = first_test(codebook, hh.N, x0, x1, y0, y1, lane, buf);
+  int cnt = n;
+  if (n <= kListMax) {
+    cnt = 0;
+    for (int k = lane; k < n; k += 32) cnt += beaten(codebook, buf, n, k, x0, x1, y0, y1) ? 0 : 1;
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
   if (lane == 0) offsets[cell + 1] = (uint32_t)cnt;
 }
 
@@ -181,22 +246,35 @@ __global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint3
   }
 }
 
-__global__ void table_fill_kernel(const float *codebook, const SearchHeader *h, const uint32_t *offsets,
-                                  uint16_t *cand) {
+__global__ void __launch_bounds__(kListThreads) table_fill_kernel(const float *codebook, const SearchHeader *h,
+                                                                  const uint32_t *offsets, uint16_t *cand) {
+  __shared__ uint16_t bufs[kListThreads / 32][kListMax];
   const int lane = threadIdx.x & 31;
+  uint16_t *buf = bufs[threadIdx.x >> 5];
   const int cell = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
   const SearchHeader hh = *h;
   if (!hh.valid || cell >= hh.G * hh.G) return;
   double x0, x1, y0, y1;
   cell_bounds(hh, cell, x0, x1, y0, y1);
-  const double bound = cell_bound(codebook, hh.N, x0, x1, y0, y1, lane);
+  const int n = first_test(codebook, hh.N, x0, x1, y0, y1, lane, buf);
   uint32_t pos = offsets[cell];
-  for (int base = 0; base < hh.N; base += 32) {
-    const int i = base + lane;
-    const bool keep = i < hh.N && dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
-    const uint32_t m = __ballot_sync(0xffffffffu, keep);
-    if (keep) cand[pos + __popc(m & ((1u << lane) - 1u))] = (uint16_t)i;
-    pos += __popc(m);
+  if (n <= kListMax) {
+    for (int base = 0; base < n; base += 32) {
+      const int k = base + lane;
+      const bool keep = k < n && !beaten(codebook, buf, n, k, x0, x1, y0, y1);
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      if (keep) cand[pos + __popc(m & ((1u << lane) - 1u))] = buf[k];
+      pos += __popc(m);
+    }
+  } else {   // too long to prune: the whole first-test list
+    const double bound = cell_bound(codebook, hh.N, x0, x1, y0, y1, lane);
+    for (int base = 0; base < hh.N; base += 32) {
+      const int i = base + lane;
+      const bool keep = i < hh.N && dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      if (keep) cand[pos + __popc(m & ((1u << lane) - 1u))] = (uint16_t)i;
+      pos += __popc(m);
+    }
   }
 }
 
@@ -211,7 +289,7 @@ cudaError_t launch_build_search_table(const float *codebook, int N, void *table,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int cells = G * G;
-  const int threads = 256;
+  const int threads = kListThreads;
   const int blocks = (cells * 32 + threads - 1) / threads;
   table_count_kernel<<<blocks, threads, 0, s>>>(codebook, h, offsets);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
