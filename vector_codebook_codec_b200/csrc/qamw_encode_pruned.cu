@@ -73,6 +73,9 @@ struct PrunedSearch {
       if (e - j > 1) {
         const float2 c0 = cb2[bi];
         float best = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
+        // one to a few iterations: not unrolled (an unrolled body with its
+        // remainder loop measured 6 us slower on the 4096^2 projection)
+#pragma unroll 1
         for (++j; j < e; ++j) {
           const int i0 = lst[j];
           const float2 c = cb2[i0];
