@@ -143,3 +143,36 @@ def test_pruned_full_size_projection_matches_oracle():
     idx, gap, _, _ = oracle_encode_rows(W, act, spec.alpha, spec.block, spec.seed, sig_o, C, rows)
     hard, _ = index_parity(e_pruned.packed.cpu().numpy().view(np.uint32)[rows], idx, gap, spec.bits)
     assert hard == 0
+
+
+def test_lists_are_pruned_subsets_of_the_first_test():
+    """The second (corner-dominance) test only removes centroids: every cell's
+    list is inside the first-test list (recomputed here in numpy with a
+    slightly larger slack, so fp64 contraction differences cannot matter), and
+    on the shipped N = 2048 codebook it removes at least a fifth of the
+    entries (about a third in practice)."""
+    N = 2048
+    C = qamw.load_codebook(N).astype(np.float64)
+    t = _read_table(qamw.build_search_table(torch.from_numpy(C.astype(np.float32)).cuda()))
+    G, off, cand = t["G"], t["offsets"], t["cand"]
+    a, UL, inv = float(t["a"]), float(t["UL"]), float(t["inv"])
+    cw = 1.0 / inv
+    k = np.arange(G)
+    lo_u, hi_u = k * cw - UL - 1e-3 * cw, (k + 1) * cw - UL + 1e-3 * cw
+    lo, hi = a * lo_u / (1 - np.abs(lo_u)), a * hi_u / (1 - np.abs(hi_u))
+    lo, hi = lo - 1e-12 * np.abs(lo), hi + 1e-12 * np.abs(hi)
+    cx, cy = C[:, 0], C[:, 1]
+    ax = np.maximum(np.abs(cx[None] - lo[:, None]), np.abs(cx[None] - hi[:, None]))      # [G, N]
+    ay = np.maximum(np.abs(cy[None] - lo[:, None]), np.abs(cy[None] - hi[:, None]))
+    bx = np.maximum(0, np.maximum(lo[:, None] - cx[None], cx[None] - hi[:, None]))
+    by = np.maximum(0, np.maximum(lo[:, None] - cy[None], cy[None] - hi[:, None]))
+    first_total = 0
+    for iy in range(G):
+        bound = (ax ** 2 + ay[iy][None] ** 2).min(axis=1) * (1 + 2e-5)                   # [G]
+        inside = (bx ** 2 + by[iy][None] ** 2) <= bound[:, None]                           # [G, N]
+        first_total += int(inside.sum())
+        for ix in range(G):
+            c = iy * G + ix
+            lst = cand[off[c]:off[c + 1]]
+            assert np.all(inside[ix, lst]), (ix, iy)
+    assert t["total"] <= 0.8 * first_total, (t["total"], first_total)
