@@ -96,7 +96,10 @@ int qamw_channel_scale(const float *act_rms, float alpha, int64_t K, float *s_ou
                        int32_t *status, qamw_stream_t stream);
 
 /*
- * qamw_calibrate_workspace_bytes -- scratch needed by qamw_calibrate_sigma.
+ * qamw_calibrate_workspace_bytes -- scratch needed by qamw_calibrate_sigma
+ * (and qamw_calibrate_partial_sums, qamw_calibrate_encode): s_j [K] and r_i
+ * [M] in fp32, then the fp64 partial sums of |z| [ceil(M/28)][K/2], each
+ * section 256-byte aligned. 0 for M < 1 or K < 2.
  */
 size_t qamw_calibrate_workspace_bytes(int64_t M, int64_t K);
 
