@@ -42,6 +42,11 @@ FALLBACK_HBM_GBS = 6650.0
 SM_COUNT_B200 = 148
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + written) of one encode_pruned_kernel launch, from the ncu
+# capture in profiles/encode_pruned_kernel_4096x4096_bf16_N2048.md (default
+# workload only). Valid while that kernel is unchanged; set to None after a
+# change until it is captured again.
+ENCODE_TRAFFIC_BYTES = {"llama7b_attn": 34437120 + 123648}
 
 
 def parse_args(argv=None):
@@ -863,7 +868,11 @@ def run_ours(args):
         evals = pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec)
         ops = 4.0 * evals
         enc_roof = {"bound": "alu", "achieved": ops / (enc_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
-                    "unit": "Gop/s", "frac": ops / (enc_ms * 1e-3) / fp32_peak, "traffic": None,
+                    "unit": "Gop/s", "frac": ops / (enc_ms * 1e-3) / fp32_peak,
+                    "traffic": ENCODE_TRAFFIC_BYTES.get(args.workload),
+                    "traffic_note": "DRAM bytes per encode_pruned_kernel launch from one ncu capture "
+                                    "(profiles/); the algorithmic bytes are the weights read and the "
+                                    "packed words written",
                     "kernel": "encode_pruned_kernel (exact pruned search; events span the qamw_encode call)",
                     "evaluations_per_pair": evals / P, "peak_source": fp32_src,
                     "brute_force_equivalent_frac": 4.0 * P * spec.N / (enc_ms * 1e-3) / fp32_peak,
