@@ -56,11 +56,15 @@ def test_status_strings(lib):
 
 
 def test_calibrate_workspace_bytes(lib):
-    M, K = 4096, 4096
-    n = lib.qamw_calibrate_workspace_bytes(M, K)
-    groups = (M + 27) // 28
-    assert n >= groups * (K // 2) * 8 + 4 * M + 4 * K
+    """The layout the header states: s [K] and r [M] in fp32, then the fp64
+    partial sums [ceil(M/28)][K/2], each section rounded up to 256 bytes."""
+    def a256(n):
+        return (n + 255) // 256 * 256
+    for M, K in ((4096, 4096), (1, 2), (29, 1000), (11008, 4096), (4096, 11008)):
+        groups = (M + 27) // 28
+        assert lib.qamw_calibrate_workspace_bytes(M, K) == a256(4 * K) + a256(4 * M) + a256(groups * (K // 2) * 8)
     assert lib.qamw_calibrate_workspace_bytes(0, 8) == 0
+    assert lib.qamw_calibrate_workspace_bytes(8, 1) == 0
 
 
 def _enc(lib, **kw):
