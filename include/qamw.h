@@ -19,8 +19,10 @@
  * matrix, shared by all rows).
  *
  * Conventions shared by every entry point
- *   - Every array pointer is a DEVICE pointer owned by the caller; the library
- *     keeps no allocation and no global state between calls.
+ *   - Every array pointer is a DEVICE pointer owned by the caller. The
+ *     library allocates nothing; between calls it keeps only caches of device
+ *     attributes (SM count, shared-memory opt-in) and the fixed scratch area
+ *     of qamw_calibrate_sigma_noalloc, none of which affects results.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and return once the kernels are enqueued.
  *   - Arguments are validated on the host before anything is launched; on a
