@@ -88,20 +88,32 @@ def lloyd(samples: np.ndarray, init: np.ndarray, max_iter: int = 500):
 # polar baseline
 # ---------------------------------------------------------------------------
 
-def lloyd_1d(values: np.ndarray, levels: int, max_iter: int = 1000) -> np.ndarray:
-    """1D Lloyd-Max quantizer levels for ``values`` (sorted ascending)."""
+def lloyd_1d(values: np.ndarray, levels: int, max_iter: int = 1_000_000) -> np.ndarray:
+    """1D Lloyd-Max quantizer levels for ``values`` (ascending).
+
+    Lloyd-Max conditions: every level is the mean of its cell, and the cells
+    meet at the midpoints between consecutive levels (a value on a midpoint
+    belongs to the lower cell). Starting from the ``levels`` quantiles of the
+    values, the two conditions are applied in turn until the partition of the
+    (sorted) values no longer changes; the levels are then the exact means of
+    their cells. A cell that empties keeps its level. The values are sorted
+    once, so each cell is a contiguous range and its sum a difference of
+    prefix sums.
+    """
     v = np.sort(np.asarray(values, dtype=np.float64))
+    S = np.concatenate([[0.0], np.cumsum(v)])
     q = np.quantile(v, (np.arange(levels) + 0.5) / levels)
+    bounds = None
     for _ in range(max_iter):
         edges = (q[1:] + q[:-1]) / 2
-        cell = np.searchsorted(edges, v)
-        cnt = np.bincount(cell, minlength=levels)
-        s = np.bincount(cell, weights=v, minlength=levels)
-        nq = np.where(cnt > 0, s / np.maximum(cnt, 1), q)
-        if np.allclose(nq, q, rtol=0, atol=1e-13):
-            q = nq
+        # cell i holds the values in (edges[i-1], edges[i]]
+        b = np.concatenate([[0], np.searchsorted(v, edges, side="right"), [v.size]])
+        if bounds is not None and np.array_equal(b, bounds):
             break
-        q = nq
+        bounds = b
+        cnt = b[1:] - b[:-1]
+        s = S[b[1:]] - S[b[:-1]]
+        q = np.where(cnt > 0, s / np.maximum(cnt, 1), q)
     return np.sort(q)
 
 

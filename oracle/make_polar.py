@@ -38,8 +38,9 @@ def main(argv):
         np.save(os.path.join(OUT_DIR, f"qamw_polar_N{N}_points.npy"), code.points().astype(np.float32))
         e["polar_amps_file"] = f"qamw_polar_N{N}_amps.npy"
         e["polar_points_file"] = f"qamw_polar_N{N}_points.npy"
-        e["polar_train_distortion_check"] = code.distortion(x)
-        print(N, A, P, e["polar_train_distortion"], e["polar_train_distortion_check"], flush=True)
+        e["polar_train_distortion"] = code.distortion(x)
+        e.pop("polar_train_distortion_check", None)
+        print(N, A, P, e["polar_train_distortion"], flush=True)
     with open(man_path, "w") as f:
         json.dump(manifest, f, indent=1, sort_keys=True)
 
