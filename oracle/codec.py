@@ -174,6 +174,12 @@ def calibrate_sigma(W, act_rms, alpha, block, seed) -> np.ndarray:
     A pair position that is zero in every row gets sigma = 1.
     """
     _, _, Y = rotated_rows(W, act_rms, alpha, block, seed)
+    return sigma_from_rotated(Y)
+
+
+def sigma_from_rotated(Y: np.ndarray) -> np.ndarray:
+    """The estimate of :func:`calibrate_sigma` from the rotated unit rows Y
+    (fp64 [M, K]): sigma_k = RN32(sqrt(2/pi) * mean_i |z_ik|), 0 -> 1."""
     Z = pairs(Y)
     amp = np.sqrt(Z[..., 0] ** 2 + Z[..., 1] ** 2)
     sig = rn32(SQRT_2_OVER_PI * (np.sum(amp, axis=0) / Z.shape[0]))
@@ -222,6 +228,61 @@ def nearest_centroid(X: np.ndarray, C: np.ndarray, chunk: int = 1 << 14):
             g = np.ones_like(d1)
         idx[a:a + chunk] = i
         gap[a:a + chunk] = g
+    return idx.reshape(shape), gap.reshape(shape)
+
+
+def nearest_centroid_kd(X: np.ndarray, C: np.ndarray, k: int = 4, chunk: int = 1 << 18):
+    """:func:`nearest_centroid` for large inputs: the same (idx, gap), bit for bit.
+
+    A k-d tree over the centroids (``scipy.spatial.cKDTree``, an exact
+    Euclidean k-nearest query used as a library primitive) proposes each
+    point's k nearest centroids. Their squared distances are recomputed with
+    the fp64 direct-difference formula of :func:`nearest_centroid`; the least
+    one (lowest index among equal distances) and the second least give idx and
+    gap. A centroid the tree did not propose is at least as far as the k-th
+    proposed one, so the answer is exact whenever the second-least recomputed
+    distance lies clearly (1e-9 relative) below the k-th; any other point, and
+    any non-finite one, is resolved by :func:`nearest_centroid`. Chunks of
+    points run on a thread pool (the tree query and numpy release the GIL).
+    """
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    from scipy.spatial import cKDTree
+    X = np.asarray(X, dtype=np.float32)
+    C64 = np.asarray(C, dtype=np.float32).astype(np.float64)
+    N = C64.shape[0]
+    if N <= k + 1:
+        return nearest_centroid(X, C)
+    shape = X.shape[:-1]
+    flat = X.reshape(-1, 2)
+    n = flat.shape[0]
+    idx = np.empty(n, dtype=np.int64)
+    gap = np.empty(n, dtype=np.float64)
+    tree = cKDTree(C64)
+
+    def run(a):
+        x = flat[a:a + chunk].astype(np.float64)
+        finite = np.all(np.isfinite(x), axis=1)
+        _, cand = tree.query(np.where(finite[:, None], x, 0.0), k=k)
+        d = (x[:, 0:1] - C64[cand, 0]) ** 2 + (x[:, 1:2] - C64[cand, 1]) ** 2
+        d1 = d.min(axis=1)
+        first = np.where(d == d1[:, None], cand, N).min(axis=1)          # lowest index at the least distance
+        d_rest = np.where(cand == first[:, None], np.inf, d)
+        d2 = d_rest.min(axis=1)
+        dk = d.max(axis=1)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            g = np.where(d2 > 0, (d2 - d1) / d2, 0.0)
+        ok = finite & (d2 < dk * (1.0 - 1e-9))
+        if not np.all(ok):
+            bad = np.nonzero(~ok)[0]
+            bi, bg = nearest_centroid(flat[a + bad], C)
+            first[bad] = bi
+            g[bad] = bg
+        idx[a:a + x.shape[0]] = first
+        gap[a:a + x.shape[0]] = g
+
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        list(ex.map(run, range(0, n, chunk)))
     return idx.reshape(shape), gap.reshape(shape)
 
 

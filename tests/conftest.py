@@ -37,3 +37,28 @@ def lib():
     from vector_codebook_codec_b200 import build, load_library
     build.build()
     return load_library()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Prints the index-parity counts the GPU tests recorded (pairs compared,
+    near ties, hard and near-tie mismatches), and writes them as JSON to the
+    file named by QAMW_PARITY_REPORT if that variable is set."""
+    pu = sys.modules.get("parity_utils")
+    recs = getattr(pu, "PARITY_RECORDS", None) if pu is not None else None
+    if not recs:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "index parity against the oracle")
+    tr.write_line(f"{'case':44s} {'scope':>14s} {'pairs':>11s} {'near-tie':>9s} {'hard':>5s} {'near-mis':>8s}")
+    tot = [0, 0, 0, 0]
+    for r in recs:
+        tr.write_line(f"{r['case'][:44]:44s} {r['scope'][:14]:>14s} {r['pairs']:11d} {r['near_tie_pairs']:9d} "
+                      f"{r['hard_mismatches']:5d} {r['near_tie_mismatches']:8d}")
+        for i, k in enumerate(("pairs", "near_tie_pairs", "hard_mismatches", "near_tie_mismatches")):
+            tot[i] += r[k]
+    tr.write_line(f"{'total':44s} {'':>14s} {tot[0]:11d} {tot[1]:9d} {tot[2]:5d} {tot[3]:8d}")
+    path = os.environ.get("QAMW_PARITY_REPORT")
+    if path:
+        import json
+        with open(path, "w") as f:
+            json.dump(recs, f, indent=1)

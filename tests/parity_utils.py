@@ -48,6 +48,12 @@ def gpu_codec(Wd, act, alpha, block, seed, C, bits, sigma=None, search="brute"):
     }
 
 
+# Index-parity records of this session: one dict per compared encoding
+# (printed at the end of the run by conftest.py, and written as JSON to the
+# file named by QAMW_PARITY_REPORT if that variable is set).
+PARITY_RECORDS: list = []
+
+
 def index_parity(gpu_packed, ora_idx, ora_gap, bits):
     """(hard mismatches, near-tie mismatches) between GPU packed rows and oracle indices."""
     P = ora_idx.shape[1]
@@ -55,6 +61,17 @@ def index_parity(gpu_packed, ora_idx, ora_gap, bits):
     diff = g != ora_idx
     near = diff & (ora_gap < TIE_GAP)
     return int(np.sum(diff & ~near)), int(np.sum(near))
+
+
+def record_parity(name, ora_gap, hard, near, scope="all pairs"):
+    """Keeps the counts of one index comparison: pairs compared, pairs whose two
+    best centroid distances are within the 1e-6 relative gap, and the hard and
+    near-tie mismatches."""
+    rec = {"case": name, "scope": scope, "pairs": int(ora_gap.size),
+           "near_tie_pairs": int(np.sum(ora_gap < TIE_GAP)), "hard_mismatches": int(hard),
+           "near_tie_mismatches": int(near)}
+    PARITY_RECORDS.append(rec)
+    return rec
 
 
 def row_scaled_error(gpu: np.ndarray, ora: np.ndarray) -> float:

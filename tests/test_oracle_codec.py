@@ -215,3 +215,30 @@ def test_zero_row_codes_nearest_to_origin_and_decodes_to_zero():
     assert np.all(enc["idx"][0] == i0)
     What = codec.decode(enc["packed"], enc["r"], sig, None, 0.0, 8, 4, 1, C, 4)
     assert np.all(What[0] == 0.0)
+
+
+@pytest.mark.parametrize("N", [2, 9, 16, 256, 2048])
+def test_kd_nearest_equals_brute_force(N):
+    """oracle.codec.nearest_centroid_kd gives the brute-force search's index
+    and gap bit for bit: Gaussian points, far points, points on centroids,
+    exact midpoints between centroid pairs (ties, lowest index wins), zeros."""
+    C = load_codebook(N) if N in (16, 256, 2048) else \
+        np.random.default_rng(N).standard_normal((N, 2)).astype(np.float32)
+    rng = np.random.default_rng(7 + N)
+    mids = ((C[rng.integers(0, N, 3000)].astype(np.float64) + C[rng.integers(0, N, 3000)]) / 2).astype(np.float32)
+    X = np.concatenate([rng.standard_normal((50000, 2)).astype(np.float32),
+                        (rng.standard_normal((2000, 2)) * 40).astype(np.float32),
+                        C[rng.integers(0, N, 2000)], mids, np.zeros((10, 2), np.float32),
+                        np.array([[np.inf, 0.0], [np.nan, 1.0]], np.float32)])
+    with np.errstate(invalid="ignore"):
+        i1, g1 = codec.nearest_centroid(X, C)
+        i2, g2 = codec.nearest_centroid_kd(X, C, chunk=4096)
+    assert np.array_equal(i1, i2)
+    assert np.array_equal(g1, g2, equal_nan=True)
+    # a symmetric codebook: many exact ties between mirrored centroids
+    Cs = np.array([[1, 0], [-1, 0], [0, 1], [0, -1], [2, 2], [-2, -2], [2, -2], [-2, 2], [3, 0], [0, 3],
+                   [-3, 0], [0, -3]], np.float32)
+    Xs = np.concatenate([np.zeros((4, 2), np.float32), rng.integers(-3, 4, (4000, 2)).astype(np.float32) / 2])
+    i1, g1 = codec.nearest_centroid(Xs, Cs)
+    i2, g2 = codec.nearest_centroid_kd(Xs, Cs, k=4)
+    assert np.array_equal(i1, i2) and np.array_equal(g1, g2)

@@ -81,7 +81,20 @@ def test_noalloc_matches_workspace_version_on_consecutive_calls(lib):
 def test_noalloc_rejects_shapes_beyond_its_area(lib):
     M, K = 8192, 8192                         # needs ~10 MiB of scratch
     assert lib.qamw_calibrate_workspace_bytes(M, K) > 8 << 20
-    rc = lib.qamw_calibrate_sigma_noalloc(ctypes.c_void_p(0x10000), QAMW_BF16, M, K, K, None, 0.5, 128, 1,
-                                          ctypes.c_void_p(0x10000), None, None)
+    W = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    sig = torch.full((K // 2,), float("nan"), dtype=torch.float32, device="cuda")
+    rc = lib.qamw_calibrate_sigma_noalloc(_p(W), QAMW_BF16, M, K, K, None, 0.5, 128, 1, _p(sig), None, _stream())
     assert rc == QAMW_EUNSUPPORTED
     assert b"built-in area" in lib.qamw_last_error()
+    torch.cuda.synchronize()
+    assert torch.isnan(sig).all()             # nothing was launched
+
+
+def test_noalloc_limit_is_the_workspace_size_rule(lib):
+    """The documented rule: align256(4K) + align256(4M) + align256(ceil(M/28) * K/2 * 8)."""
+    def need(M, K):
+        a = lambda v: (v + 255) // 256 * 256
+        return a(4 * K) + a(4 * M) + a(-(-M // 28) * (K // 2) * 8)
+    for M, K in [(1, 2), (1, 1 << 21), (27, 4096), (28, 4096), (4096, 4096), (11008, 4096), (5, 10)]:
+        assert lib.qamw_calibrate_workspace_bytes(M, K) == need(M, K)
+    assert need(1, 1 << 21) > 8 << 20 and need(4096, 4096) <= 8 << 20
