@@ -159,13 +159,19 @@ int qamw_sigma_from_partial_sums(const double *sums, int32_t R, int64_t P, int64
  * workspace, using a fixed scratch area of QAMW_NOALLOC_SCRATCH_BYTES bytes
  * built into the library; neither it nor the library allocates anything.
  *   - Limit: qamw_calibrate_workspace_bytes(M, K) must not exceed
- *     QAMW_NOALLOC_SCRATCH_BYTES (about M*K <= 58 million weights);
- *     larger shapes return QAMW_EUNSUPPORTED with a message that says so.
+ *     QAMW_NOALLOC_SCRATCH_BYTES, i.e.
+ *       align256(4K) + align256(4M) + align256(ceil(M/28) * (K/2) * 8) <= 8 MiB
+ *     (align256 rounds up to a multiple of 256). For large M this is about
+ *     M*K <= 58 million weights; for M < 28 the partial sums alone take 4K
+ *     bytes, so K is at most about 2 million. Larger shapes return
+ *     QAMW_EUNSUPPORTED with a message that says so.
  *   - The area is reserved on every GPU that loads the library, until the
  *     process exits.
- *   - Set-up: the first call made with a given device current looks up the
- *     area's device address (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture on that device.
+ *   - Set-up: the first call made in a given context (device) looks up the
+ *     area's device address (cudaGetSymbolAddress) and caches it with that
+ *     context; a call in another context (after cudaDeviceReset, or with a
+ *     non-primary context current) looks it up again. Make the first call
+ *     in a context before any stream capture in it.
  *   - All calls share the one area and it keeps the last call's contents;
  *     nothing in it needs to start at zero (each call writes every byte it
  *     reads). Calls whose kernels overlap on the GPU (different streams, or

@@ -13,10 +13,15 @@
 // The area is a file-scope device array of QAMW_NOALLOC_SCRATCH_BYTES bytes;
 // every GPU that loads the library reserves it until the process exits. In
 // host code its name is only a handle for the symbol, not a device address,
-// so the address is looked up once per device with cudaGetSymbolAddress (on
-// the first call made with that device current) and cached.
+// so the address is looked up with cudaGetSymbolAddress (on the first call
+// made with a device current) and cached. The cache entry remembers the
+// driver context it was looked up in: after cudaDeviceReset, or with another
+// context current on the same device, the module is loaded anew at another
+// address, so a call in a new context looks the address up again.
 #include <cstdio>
 #include <mutex>
+
+#include <cuda.h>
 
 #include "qamw.h"
 #include "qamw_internal.h"
@@ -27,22 +32,48 @@ static __device__ __align__(256) unsigned char g_calib_scratch[QAMW_NOALLOC_SCRA
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+struct ScratchEntry {
+  CUcontext ctx;
+  void *addr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of this module's scratch area on the current device.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+// The driver's cuCtxGetCurrent, reached through the runtime (no -lcuda).
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of this module's scratch area in the current context.
 cudaError_t scratch_address(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr) return cudaErrorDeviceUninitialized;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;   // NULL before the runtime's first use
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchEntry &ent = g_scratch[dev];
+  if (ctx == nullptr || ent.addr == nullptr || ent.ctx != ctx) {
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_calib_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    if ((e = cudaGetSymbolAddress(&p, g_calib_scratch)) != cudaSuccess) return e;   // sets a context current
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+    ent.ctx = ctx;
+    ent.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = ent.addr;
   return cudaSuccess;
 }
 
