@@ -254,6 +254,19 @@ int qamw_build_search_table(const float *codebook, int32_t N, void *table, size_
                             qamw_stream_t stream);
 
 /*
+ * qamw_search_cells -- test hook for the pruned search of Methodology (4):
+ * the grid cell the encode assigns to each normalised pair, computed by the
+ * encode's own device function (cell_out[i] = iy * G + ix of the table's
+ * grid, or -1 for a pair outside the grid or an invalid table). With the
+ * table's lists it lets a test check that every pair's exact nearest
+ * centroid is listed in the cell the encode actually looks in.
+ * (An interface of this library; the QAM-W page has no counterpart.)
+ *   x: device float32 [n][2]   table: as for qamw_encode   cell_out: device int32 [n]
+ * Errors: QAMW_ENULL, QAMW_EINVAL (n < 0, table not 16-byte aligned).
+ */
+int qamw_search_cells(const float *x, int64_t n, const void *table, int32_t *cell_out, qamw_stream_t stream);
+
+/*
  * qamw_encode_polar -- the polar baseline codec ("Joint 2D vs. Polar", Results
  * of the QAM-W page): steps (5), (1), (2), (3) exactly as qamw_encode, then
  * the amplitude and the phase of each normalised pair are quantized

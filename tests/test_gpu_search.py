@@ -20,19 +20,35 @@ def _built(lib):
     return lib
 
 
-HEADER_BYTES = 48
+IMAGE_OFFSET = 64
 
 
 def _read_table(table):
+    """Header fields and every cell's list (offsets/cand, concatenated in cell
+    order) decoded from the table's records and overflow lists."""
     raw = table.cpu().numpy()
-    hdr = raw[:HEADER_BYTES].view(np.int32)
+    hdr = raw[:48].view(np.int32)
     magic, N, G, total, valid, cap = (int(hdr[0]) & 0xFFFFFFFF, int(hdr[1]), int(hdr[2]), int(hdr[3]),
                                       int(hdr[4]), int(hdr[5]))
     a, UL, inv, L = raw[24:40].view(np.float32)
-    offsets = raw[HEADER_BYTES:HEADER_BYTES + 4 * (G * G + 1)].view(np.uint32).astype(np.int64)
-    cand = raw[HEADER_BYTES + 4 * (G * G + 1):].view(np.uint16)[:total].astype(np.int64)
+    rec = raw[IMAGE_OFFSET:IMAGE_OFFSET + 8 * G * G].view(np.uint64)
+    ovf = raw[IMAGE_OFFSET + 8 * G * G:].view(np.uint16).astype(np.int64)
+    e = np.stack([(rec >> np.uint64(16 * f)) & np.uint64(0xFFFF) for f in range(3)], axis=1).astype(np.int64)
+    meta = (rec >> np.uint64(48)).astype(np.int64)
+    n = meta & 3
+    lists = []
+    for c in range(G * G):
+        if n[c] > 0:
+            lists.append(e[c, :n[c]])
+        else:
+            o = meta[c] >> 2
+            lists.append(np.concatenate([e[c], ovf[o + 1:o + 1 + ovf[o]]]))
+    lens = np.array([x.size for x in lists], dtype=np.int64)
+    offsets = np.concatenate([[0], np.cumsum(lens)])
+    cand = np.concatenate(lists)
     return dict(magic=magic, N=N, G=G, total=total, valid=valid, capacity=cap, a=np.float32(a),
-                UL=np.float32(UL), inv=np.float32(inv), L=float(L), offsets=offsets, cand=cand)
+                UL=np.float32(UL), inv=np.float32(inv), L=float(L), offsets=offsets, cand=cand, records=rec,
+                n_inline=n)
 
 
 def _cell_coord(x, t):
@@ -49,7 +65,7 @@ def test_table_lists_the_nearest_centroid_of_every_point(N):
     assert t["valid"] == 1 and t["N"] == N
     G, L, off, cand = t["G"], t["L"], t["offsets"], t["cand"]
     assert L > np.abs(C).max()
-    assert off[0] == 0 and off[-1] == t["total"] and np.all(np.diff(off) >= 1)
+    assert off[0] == 0 and np.all(np.diff(off) >= 1) and t["total"] <= t["capacity"]
     for k in range(G * G):
         lst = cand[off[k]:off[k + 1]]
         assert np.all(np.diff(lst) > 0) and lst.max() < N
@@ -124,7 +140,9 @@ def test_pruned_outside_grid_points():
     assert torch.equal(a.packed, b.packed)
 
 
-def test_pruned_full_size_projection_matches_oracle():
+def test_pruned_full_size_projection_equals_brute_force():
+    """Whole 4096x4096 projection: pruned and brute-force packed streams are
+    identical (test_gpu_fullsize compares every pair with the oracle)."""
     spec = synth.llama7b_attn().specs[0]
     w32 = synth.make_matrix(spec)
     act = synth.act_for(spec)
@@ -138,11 +156,46 @@ def test_pruned_full_size_projection_matches_oracle():
     e_pruned = qamw.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sig, Cd, spec.bits, search_table=table)
     torch.cuda.synchronize()
     assert torch.equal(e_brute.packed, e_pruned.packed)
-    sig_o = codec.calibrate_sigma(W, act, spec.alpha, spec.block, spec.seed)
-    rows = np.array([0, 1, 2047, spec.M - 1])
-    idx, gap, _, _ = oracle_encode_rows(W, act, spec.alpha, spec.block, spec.seed, sig_o, C, rows)
-    hard, _ = index_parity(e_pruned.packed.cpu().numpy().view(np.uint32)[rows], idx, gap, spec.bits)
-    assert hard == 0
+
+
+@pytest.mark.parametrize("N", [16, 128, 256, 1024, 2048])
+def test_cells_the_encode_computes_list_the_nearest_centroid(N):
+    """The encode's own cell arithmetic (qamw_search_cells runs its device
+    function): for points on and within 1e-4 cells of every kind of cell edge,
+    the cell the encode looks in lists the oracle's nearest centroid; and that
+    cell is the exact cell (fp64) or, within 1e-3 cells of an edge, a
+    neighbour whose enlarged bounds contain the point."""
+    C = qamw.load_codebook(N)
+    Cd = torch.from_numpy(C).cuda()
+    table = qamw.build_search_table(Cd)
+    t = _read_table(table)
+    G, off, cand = t["G"], t["offsets"], t["cand"]
+    assert G % 2 == 1
+    a, UL, inv = float(t["a"]), float(t["UL"]), float(t["inv"])
+    rng = np.random.default_rng(1000 + N)
+    n = 200000
+    k = rng.integers(0, G + 1, size=(n, 2)).astype(np.float64)
+    jitter = np.where(rng.random((n, 2)) < 0.2, 0.0, rng.uniform(-1e-4, 1e-4, size=(n, 2)))
+    u = np.clip((k + jitter) / inv - UL, -0.9999, 0.9999)
+    pts = (a * u / (1.0 - np.abs(u))).astype(np.float32)
+    pts = np.concatenate([pts, rng.standard_normal((n, 2)).astype(np.float32)])
+    cells = qamw.search_cells(torch.from_numpy(pts).cuda(), table).cpu().numpy().astype(np.int64)
+    inside = cells >= 0
+    assert inside.mean() > 0.9
+    # exact (fp64) cell coordinates; the encode's must agree up to 1e-3 cells
+    p64 = pts.astype(np.float64)
+    f = (p64 / (a + np.abs(p64)) + UL) * inv
+    cx, cy = cells % G, cells // G
+    for c, ff in ((cx, f[:, 0]), (cy, f[:, 1])):
+        sel = inside
+        assert np.all((ff[sel] >= c[sel] - 1e-3) & (ff[sel] <= c[sel] + 1 + 1e-3))
+    idx, _ = codec.nearest_centroid_kd(pts[inside], C)
+    for c, i in zip(cells[inside], idx):
+        assert i in cand[off[c]:off[c + 1]]
+    # points beyond the grid, huge and non-finite ones are off the grid
+    far = np.array([[t["L"] * 1.01, 0], [0, -t["L"] * 1.01], [1e38, 0], [3e38, -3e38], [np.nan, 0],
+                    [np.inf, 1]], np.float32)
+    assert np.all(qamw.search_cells(torch.from_numpy(far).cuda(), table).cpu().numpy() == -1)
 
 
 def test_lists_are_pruned_subsets_of_the_first_test():
@@ -175,4 +228,29 @@ def test_lists_are_pruned_subsets_of_the_first_test():
             c = iy * G + ix
             lst = cand[off[c]:off[c + 1]]
             assert np.all(inside[ix, lst]), (ix, iy)
-    assert t["total"] <= 0.8 * first_total, (t["total"], first_total)
+    assert off[-1] <= 0.8 * first_total, (off[-1], first_total)
+
+
+def test_records_hold_short_lists_inline():
+    """The table layout: a list of one to three entries sits in its cell's
+    record (unused fields repeat the first entry); longer lists keep their
+    first three entries inline and the rest, counted, in the overflow array,
+    which holds nothing else."""
+    C = qamw.load_codebook(2048)
+    t = _read_table(qamw.build_search_table(torch.from_numpy(C).cuda()))
+    n, rec = t["n_inline"], t["records"]
+    off, cand = t["offsets"], t["cand"]
+    lens = np.diff(off)
+    assert np.array_equal(np.where(n > 0, n, 0), np.where(lens <= 3, lens, 0))
+    e0 = (rec & np.uint64(0xFFFF)).astype(np.int64)
+    for f in (1, 2):
+        ef = ((rec >> np.uint64(16 * f)) & np.uint64(0xFFFF)).astype(np.int64)
+        short = (lens >= 1) & (lens <= f)
+        assert np.array_equal(ef[short], e0[short])
+    long_ = lens > 3
+    assert t["total"] == int(np.sum(lens[long_] - 3 + 1))
+    # most pairs of the unit circular Gaussian fall in cells of at most three entries
+    G, a, UL, inv = t["G"], float(t["a"]), float(t["UL"]), float(t["inv"])
+    x = np.random.default_rng(5).standard_normal((200000, 2))
+    f = np.floor((x / (a + np.abs(x)) + UL) * inv).astype(np.int64)
+    assert np.mean(lens[f[:, 1] * G + f[:, 0]] <= 3) > 0.9

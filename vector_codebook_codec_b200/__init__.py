@@ -53,6 +53,7 @@ _SIGNATURES = {
     "qamw_decode": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
                                    _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
+    "qamw_search_cells": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p]),
     "qamw_search_table_bytes": (_c_sz, [_c_i32]),
     "qamw_build_search_table": (ctypes.c_int, [_c_p, _c_i32, _c_p, _c_sz, _c_p]),
     "qamw_calibrate_sigma_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
@@ -425,6 +426,18 @@ def rotate_rows(U, block: int, seed: int, inverse: bool = False, stream=None):
     _check("qamw_rotate_rows", load_library().qamw_rotate_rows(
         _ptr(U), _ptr(Y), M, K, block, seed & (2**64 - 1), 1 if inverse else 0, _stream_ptr(stream)))
     return Y
+
+
+def search_cells(x, table, stream=None):
+    """The encode's grid cell of each pair of x (float32 CUDA tensor [n, 2]) for
+    a search table (int32 tensor [n]; -1 outside the grid). Test hook."""
+    torch = _torch()
+    _need_cuda("x", x, torch.float32, 2)
+    x = x.contiguous()
+    out = torch.empty(x.shape[0], dtype=torch.int32, device=x.device)
+    _check("qamw_search_cells", load_library().qamw_search_cells(
+        _ptr(x), x.shape[0], _ptr(table), _ptr(out), _stream_ptr(stream)))
+    return out
 
 
 # ---------------------------------------------------------------------------

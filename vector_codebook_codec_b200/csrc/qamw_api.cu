@@ -437,7 +437,20 @@ int qamw_rotate_rows(const double *U, double *Y, int64_t M, int64_t K, int32_t b
   if (!U || !Y) return fail(QAMW_ENULL, "%s: U and Y must be non-NULL", fn);
   if ((rc = check_shape(M, K, block, fn))) return rc;
   RotateTestArgs a{U, Y, M, K, log2i(block), sign_seed, inverse};
-  cudaError_t e = launch_rotate_test(a, (cudaStream_t)stream);
+  cudaError_t e = (a.log2b <= 9) ? launch_rotate_test512(a, (cudaStream_t)stream)
+                                 : launch_rotate_test(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+int qamw_search_cells(const float *x, int64_t n, const void *table, int32_t *cell_out, qamw_stream_t stream) {
+  static const char *fn = "qamw_search_cells";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  if (!x || !table || !cell_out) return fail(QAMW_ENULL, "%s: x, table and cell_out must be non-NULL", fn);
+  if (n < 0) return fail(QAMW_EINVAL, "%s: n must be >= 0", fn);
+  if (n == 0) return QAMW_OK;
+  if (reinterpret_cast<uintptr_t>(table) % 16) return fail(QAMW_EINVAL, "%s: table must be 16-byte aligned", fn);
+  cudaError_t e = launch_search_cells(x, n, table, cell_out, (cudaStream_t)stream);
   return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
 }
 

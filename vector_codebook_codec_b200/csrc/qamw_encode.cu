@@ -506,10 +506,10 @@ cudaError_t launch_channel_scale(const ScaleArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_row_norms(const RowNormArgs &a, cudaStream_t s) {
-  const int threads = 256;
-  const int64_t blocks = std::min<int64_t>((a.M + 7) / 8, (int64_t)sm_count() * 8);
   const int epv = (a.wt == QAMW_BF16) ? 8 : 4;
   const int vec = (w_vec_ok(a.W, a.wt, a.ldw) && a.K % epv == 0 && reinterpret_cast<uintptr_t>(a.s) % 16 == 0) ? 1 : 0;
+  const int threads = 256;
+  const int64_t blocks = std::min<int64_t>((a.M + 7) / 8, (int64_t)sm_count() * 8);
   if (a.wt == QAMW_BF16)
     row_norm_kernel<QAMW_BF16><<<(int)blocks, threads, 0, s>>>(a, vec);
   else

@@ -50,14 +50,14 @@ struct PolarSearch {
 };
 
 template <int WT>
-__global__ void __launch_bounds__(kUnitThreads, 1) encode_polar_kernel(EncodeArgs a, int vec_ok) {
+__global__ void __launch_bounds__(kEncThreads, 1) encode_polar_kernel(EncodeArgs a, int vec_ok) {
   extern __shared__ __align__(16) unsigned char smem[];
   double *edges = reinterpret_cast<double *>(smem + kUnitSmemBytes);
   const int A1 = a.polar_A - 1;
-  for (int i = threadIdx.x; i < A1; i += kUnitThreads) edges[i] = (a.polar_amps[i] + a.polar_amps[i + 1]) * 0.5;
+  for (int i = threadIdx.x; i < A1; i += kEncThreads) edges[i] = (a.polar_amps[i] + a.polar_amps[i + 1]) * 0.5;
   // encode_units synchronises the CTA before the first pair is quantized
   const PolarSearch S{edges, A1, a.polar_P, kTwoPi / (double)a.polar_P};
-  encode_units<WT>(a, vec_ok, smem, S);
+  encode_units<WT, 0, 0>(a, vec_ok, smem, S);
 }
 
 template <int WT>
@@ -66,11 +66,11 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(encode_polar_kernel<WT>), smem);
   if (e != cudaSuccess) return e;
   const int64_t n_chunks = (a.rot.K + kUnit - 1) / kUnit;
-  const int64_t tiles = n_chunks * ((a.rot.M + kUnitWarps - 1) / kUnitWarps);
+  const int64_t tiles = n_chunks * ((a.rot.M + kEncWarps - 1) / kEncWarps);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count()));
   const size_t es = (WT == QAMW_BF16) ? 2 : 4;
   const int vec = ((reinterpret_cast<uintptr_t>(a.rot.W) % 16) == 0 && (a.rot.ldw * (int64_t)es) % 16 == 0) ? 1 : 0;
-  encode_polar_kernel<WT><<<(int)blocks, kUnitThreads, smem, s>>>(a, vec);
+  encode_polar_kernel<WT><<<(int)blocks, kEncThreads, smem, s>>>(a, vec);
   return cudaGetLastError();
 }
 

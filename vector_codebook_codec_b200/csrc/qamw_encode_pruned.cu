@@ -7,21 +7,21 @@
 // block Hadamard rotation (step 2), x = z / sigma (step 3), nearest centroid
 // (step 4) with the channel scale s_j applied first (step 5), then bit packing.
 //
-// Work decomposition. A *unit* is one row x 512 consecutive columns handled by
-// one warp: lane l owns columns [16l, 16l + 16) of the unit (8 pairs); the
-// rotation is the fp64 one of qamw_rotate16.cuh, which gives the same x bit
-// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 28 warps takes a contiguous
-// range of *tiles* (28 rows x one 512-column chunk) in chunk-major order; the
-// chunk's d_j * s_j and 1 / sigma_k live once per CTA in shared memory, next
-// to the codebook and the search table. The next unit's weights are loaded
-// while the current one is searched.
+// Work decomposition: the 512-column pipeline of qamw_encode_unit.cuh (a
+// unit is one row x 512 columns per warp, rotated in fp64 so that x is the
+// correctly rounded value; 16 warps per CTA, tiles in chunk-major order).
 //
-// Search. The pair's cell of the search table (qamw_search.cu) lists every
-// centroid that can be an fp32 minimiser, in ascending index order; a strict
-// "<" over the list keeps the lowest index among equal distances, which is the
-// brute-force result. In shared memory the lists follow an identity list
-// 0..N-1, which a pair outside the grid (or every pair, if the table does not
-// fit or does not match the codebook) scans instead.
+// Search. The pair's grid cell (search_cell, qamw_internal.h) has a record of
+// the search table (qamw_search.cu) listing, in ascending index order, every
+// centroid that can be an fp32 minimiser for a pair in the cell: up to three
+// inline, longer lists continuing in an overflow array. A one-entry list is
+// the answer without a distance; otherwise a strict "<" over the list keeps
+// the lowest index among equal distances, which is the brute-force result. A
+// pair outside the grid, or every pair if the table is invalid or does not
+// fit, scans all N centroids. The records and overflow lists are copied once
+// per CTA into shared memory with bulk asynchronous copies (one thread, an
+// mbarrier with a bounded wait); the codebook is copied from the codebook
+// argument.
 #include <algorithm>
 #include <cfloat>
 #include <cmath>
@@ -29,110 +29,142 @@
 #include "qamw_device.cuh"
 #include "qamw_internal.h"
 #include "qamw_encode_unit.cuh"
+#include "qamw_mbarrier.cuh"
 
 namespace qamw {
 namespace {
 
-constexpr int kThreads = kUnitThreads;
+constexpr int kThreads = kEncThreads;
+
 
 // The exact pruned search over the codebook's grid table (see the file comment).
 struct PrunedSearch {
   const float2 *cb2;
-  const uint16_t *toff, *lst;
+  const uint64_t *rec;
+  const uint16_t *ovf;
   bool use;
-  int G, N;
-  float a_ax, UL, inv_cw, Gf;
+  int G, N, total;
+  float a_ax, inv_cw, cbias, L;
 
   __device__ __forceinline__ void search8(const float (&x0)[8], const float (&x1)[8], int (&idx)[8]) const {
-    // candidate ranges of the 8 pairs (cell lists, or the identity list),
-    // without branches: an off-grid pair reads cell 0 and discards it
-    int beg[8], end[8];
+    // Every pair evaluates the three inline entries of its cell's record
+    // without a branch: a list of one or two repeats its first entry there,
+    // and a repeated entry never wins a strict "<". Listed entries are in
+    // ascending index order, so the strict "<" keeps the lowest index among
+    // equal distances: the brute-force result. Pairs whose list continues in
+    // the overflow array, and pairs outside the grid (whose record reads as
+    // "0, 0, 0" and continue over all N centroids), finish in a loop that the
+    // warp enters only if one of its lanes needs it.
+    float best[8];
+    int meta[8];
+    uint32_t more = 0;
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
-      const float u0 = __fdividef(x0[p], __fadd_rn(a_ax, fabsf(x0[p])));
-      const float u1 = __fdividef(x1[p], __fadd_rn(a_ax, fabsf(x1[p])));
-      const float fx = __fmul_rn(__fadd_rn(u0, UL), inv_cw);
-      const float fy = __fmul_rn(__fadd_rn(u1, UL), inv_cw);
-      const bool in = use && fx >= 0.0f && fx < Gf && fy >= 0.0f && fy < Gf;
-      const int cell = in ? (int)fy * G + (int)fx : 0;
-      const int b0 = toff[cell], e0 = toff[cell + 1];
-      beg[p] = in ? b0 : 0;
-      end[p] = in ? e0 : N;
+      const int cell = use ? search_cell(x0[p], x1[p], a_ax, inv_cw, cbias, L, G) : -1;
+      const uint2 r = cell >= 0 ? reinterpret_cast<const uint2 *>(rec)[cell] : make_uint2(0u, 0u);
+      // indices clamped below N, so that no table content can read outside the codebook
+      const int e0 = min((int)(r.x & 0xffffu), N - 1), e1 = min((int)(r.x >> 16), N - 1),
+                e2 = min((int)(r.y & 0xffffu), N - 1);
+      meta[p] = cell >= 0 ? (int)(r.y >> 16) : -1;
+      const float2 c0 = cb2[e0], c1 = cb2[e1], c2 = cb2[e2];
+      float b = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
+      int bi = e0;
+      const float d1 = dist2_scalar(x0[p], x1[p], c1.x, c1.y);
+      const float d2 = dist2_scalar(x0[p], x1[p], c2.x, c2.y);
+      if (d1 < b) { b = d1; bi = e1; }
+      if (d2 < b) { b = d2; bi = e2; }
+      best[p] = b;
+      idx[p] = bi;
+      if (meta[p] < 0 || (meta[p] & 3) == 0) more |= 1u << p;   // off the grid (meta = -1) or an overflow list
     }
-    // Every list has at least one entry. A single-entry list is the answer
-    // without a distance (30% of the pairs on the 4096^2 projection, whose
-    // lanes then issue no codebook read); otherwise the first entry's distance
-    // starts the strict "<" scan of the rest. The first entry of the identity
-    // list is index 0, so an off-grid pair whose distances all overflow to
-    // +inf still gets index 0, as in the brute-force search.
+    if (__any_sync(0xffffffffu, more != 0)) {
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      const int e = end[p];
-      int j = beg[p];
-      int bi = lst[j];
-      if (e - j > 1) {
-        const float2 c0 = cb2[bi];
-        float best = dist2_scalar(x0[p], x1[p], c0.x, c0.y);
-        // one to a few iterations: not unrolled (an unrolled body with its
-        // remainder loop measured 6 us slower on the 4096^2 projection)
+      for (int p = 0; p < 8; ++p) {
+        if (more & (1u << p)) {
+          const bool off_grid = meta[p] < 0;
+          // (clamped to the copied overflow entries)
+          const int o = min(meta[p] >> 2, total - 1);
+          const int kb = off_grid ? 0 : o + 1, ke = off_grid ? N : min(o + 1 + (int)ovf[max(o, 0)], total);
+          float b = best[p];
+          int bi = idx[p];
 #pragma unroll 1
-        for (++j; j < e; ++j) {
-          const int i0 = lst[j];
-          const float2 c = cb2[i0];
-          const float d0 = dist2_scalar(x0[p], x1[p], c.x, c.y);
-          if (d0 < best) { best = d0; bi = i0; }
+          for (int k = kb; k < ke; ++k) {
+            const int ik = off_grid ? k : min((int)ovf[k], N - 1);
+            const float2 c = cb2[ik];
+            const float d = dist2_scalar(x0[p], x1[p], c.x, c.y);
+            if (d < b) { b = d; bi = ik; }
+          }
+          idx[p] = bi;
         }
       }
-      idx[p] = bi;
     }
   }
 };
 
-template <int WT>
-__global__ void __launch_bounds__(kThreads, 1)
-    encode_pruned_kernel(EncodeArgs a, int vec_ok, int tab_cap, int toff_slots) {
+// Shared memory after the encode pipeline's: the codebook (float2 [N], from
+// the codebook argument), then the table's image (records and overflow
+// lists), copied by one thread with bulk asynchronous copies.
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+constexpr uint32_t kTableWaitLimit = 1u << 22;   // try_wait attempts for the table copy (far beyond its ~2 us)
+
+template <int WT, int LB, int BB>
+__global__ void __launch_bounds__(kThreads, 1) encode_pruned_kernel(EncodeArgs a, int vec_ok, int image_cap) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int N = a.N;
   const int n2 = (N + 1) & ~1;
   float2 *cb2 = reinterpret_cast<float2 *>(smem + kUnitSmemBytes);
-  uint16_t *toff = reinterpret_cast<uint16_t *>(cb2 + n2);
-  uint16_t *lst = toff + toff_slots;   // identity list 0..N-1, then the cell lists
+  unsigned char *image = reinterpret_cast<unsigned char *>(cb2 + n2);
 
-  __shared__ int s_use, s_G;
-  __shared__ float s_a, s_UL, s_inv;
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ int s_use, s_G, s_total;
+  __shared__ float s_a, s_inv, s_L;
   if (threadIdx.x == 0) {
     const SearchHeader h = *reinterpret_cast<const SearchHeader *>(a.table);
-    const bool ok = h.magic == kSearchMagic && h.valid == 1 && h.N == N && h.G >= 1 && h.G <= 181 &&
-                    h.G * h.G + 1 <= toff_slots && h.total >= 0 && h.total <= tab_cap - N &&
-                    h.total + N < 65536 && h.a > 0.0f && h.UL > 0.0f && h.UL < 1.0f && h.inv_cw > 0.0f;
+    const int64_t rec_bytes = (int64_t)h.G * h.G * 8;
+    const int64_t copy = (rec_bytes + 2 * (int64_t)h.total + 15) & ~(int64_t)15;
+    bool ok = h.magic == kSearchMagic && h.valid == 1 && h.N == N && h.G >= 1 && h.G <= kSearchMaxG &&
+              (h.G & 1) == 1 && h.total >= 0 && h.total <= h.capacity && copy <= h.image_bytes &&
+              copy <= (int64_t)image_cap && h.a > 0.0f && h.UL > 0.0f && h.UL < 1.0f && h.inv_cw > 0.0f &&
+              h.L > 0.0f;
+    if (ok) {
+      mbar_init(&s_bar, 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      mbar_arrive_expect_tx(&s_bar, (uint32_t)copy);
+      const unsigned char *src = reinterpret_cast<const unsigned char *>(a.table) + kSearchImageOffset;
+      for (int64_t o = 0; o < copy; o += 32768) {
+        const uint32_t nb = (uint32_t)((copy - o) < 32768 ? (copy - o) : 32768);
+        bulk_copy_g2s(image + o, src + o, nb, &s_bar);
+      }
+      if (!mbar_wait(&s_bar, 0, kTableWaitLimit)) {
+        status_or(a.status, QAMW_STATUS_TIMEOUT);
+        mbar_wait(&s_bar, 0, kTableWaitLimit);   // give the copy a second bounded chance to land
+        ok = false;
+      }
+    }
     s_use = ok ? 1 : 0;
-    s_G = h.G;
+    s_G = ok ? h.G : 1;
+    s_total = ok ? h.total : 0;
     s_a = h.a;
-    s_UL = h.UL;
     s_inv = h.inv_cw;
+    s_L = h.L;
   }
   for (int c = threadIdx.x; c < n2; c += kThreads)
     cb2[c] = (c < N) ? make_float2(a.codebook[2 * c], a.codebook[2 * c + 1]) : make_float2(0.0f, 0.0f);
-  for (int i = threadIdx.x; i < N; i += kThreads) lst[i] = (uint16_t)i;
   __syncthreads();
   const bool use = s_use != 0;
   const int G = s_G;
-  if (use) {
-    const uint32_t *goff = reinterpret_cast<const uint32_t *>(reinterpret_cast<const unsigned char *>(a.table) +
-                                                              sizeof(SearchHeader));
-    const uint16_t *gcand = reinterpret_cast<const uint16_t *>(goff + G * G + 1);
-    // clamped on the copy, so that no table content can index outside the
-    // lists or the codebook
-    const uint32_t total = goff[G * G] < (uint32_t)(tab_cap - N) ? goff[G * G] : (uint32_t)(tab_cap - N);
-    for (int i = threadIdx.x; i <= G * G; i += kThreads)
-      toff[i] = (uint16_t)((goff[i] < total ? goff[i] : total) + (uint32_t)N);
-    for (int i = threadIdx.x; i < (int)total; i += kThreads)
-      lst[N + i] = (gcand[i] < (uint16_t)N) ? gcand[i] : (uint16_t)(N - 1);
-  }
-  const float a_ax = s_a, UL = s_UL, inv_cw = s_inv, Gf = (float)G;
+  const uint64_t *rec = reinterpret_cast<const uint64_t *>(image);
+  const uint16_t *ovf = reinterpret_cast<const uint16_t *>(image + (size_t)G * G * 8);
+  const float a_ax = s_a, inv_cw = s_inv, L = s_L;
+  const float cbias = kCellMagic + (float)((G - 1) / 2);
 
-  const PrunedSearch S{cb2, toff, lst, use, G, N, a_ax, UL, inv_cw, Gf};
-  encode_units<WT>(a, vec_ok, smem, S);
+  const PrunedSearch S{cb2, rec, ovf, use, G, N, s_total, a_ax, inv_cw, cbias, L};
+  encode_units<WT, LB, BB>(a, vec_ok, smem, S);
 }
 
 template <typename Kern>
@@ -140,29 +172,41 @@ cudaError_t set_smem(Kern k, size_t bytes) {
   return set_max_dynamic_smem(reinterpret_cast<const void *>(k), bytes);
 }
 
-template <int WT>
+template <int WT, int LB, int BB>
 cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
   int dev = 0, smem_max = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-  const int G = search_grid(a.N);
-  const int toff_slots = (G * G + 1 + 7) & ~7;
   const int n2 = (a.N + 1) & ~1;
-  const size_t base = kUnitSmemBytes + (size_t)n2 * sizeof(float2) + (size_t)toff_slots * 2;
-  const int64_t room = ((int64_t)smem_max - 128 /*static*/ - (int64_t)base) / 2;
-  int tab_cap = (int)std::max<int64_t>(0, std::min<int64_t>(room, 65535));
-  tab_cap &= ~7;
-  if (tab_cap < a.N) return cudaErrorInvalidConfiguration;   // the launcher only comes here for N <= 2048
-  const size_t smem = base + (size_t)tab_cap * 2;
-  if ((e = set_smem(encode_pruned_kernel<WT>, smem)) != cudaSuccess) return e;
+  const size_t base = kUnitSmemBytes + (size_t)n2 * sizeof(float2);
+  const int64_t room = ((int64_t)smem_max - 256 /*static*/ - (int64_t)base) & ~(int64_t)15;
+  if (room < 16) return cudaErrorInvalidConfiguration;
+  // the image of the table (or as much of it as fits; a table that does not
+  // fit makes every pair take the brute-force loop)
+  const int image_cap = (int)std::min<int64_t>(room, (int64_t)search_table_bytes(a.N));
+  const size_t smem = base + (size_t)image_cap;
+  if ((e = set_smem(encode_pruned_kernel<WT, LB, BB>, smem)) != cudaSuccess) return e;
   const int64_t n_chunks = (a.rot.K + kUnit - 1) / kUnit;
-  const int64_t tiles = n_chunks * ((a.rot.M + kUnitWarps - 1) / kUnitWarps);
+  const int64_t tiles = n_chunks * ((a.rot.M + kEncWarps - 1) / kEncWarps);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count()));
   const size_t es = (WT == QAMW_BF16) ? 2 : 4;
   const int vec = ((reinterpret_cast<uintptr_t>(a.rot.W) % 16) == 0 && (a.rot.ldw * (int64_t)es) % 16 == 0) ? 1 : 0;
-  encode_pruned_kernel<WT><<<(int)blocks, kThreads, smem, s>>>(a, vec, tab_cap, toff_slots);
+  encode_pruned_kernel<WT, LB, BB><<<(int)blocks, kThreads, smem, s>>>(a, vec, image_cap);
   return cudaGetLastError();
+}
+
+// The bf16 workloads' shapes compiled for their block size (128, 256) and
+// code size (10, 11 bits); every other shape takes the run-time version.
+template <int WT>
+cudaError_t launch_wt(const EncodeArgs &a, cudaStream_t s) {
+  if (WT == QAMW_BF16) {
+    if (a.rot.log2b == 7 && a.bits == 11) return launch_t<WT, 7, 11>(a, s);
+    if (a.rot.log2b == 8 && a.bits == 11) return launch_t<WT, 8, 11>(a, s);
+    if (a.rot.log2b == 7 && a.bits == 10) return launch_t<WT, 7, 10>(a, s);
+    if (a.rot.log2b == 8 && a.bits == 10) return launch_t<WT, 8, 10>(a, s);
+  }
+  return launch_t<WT, 0, 0>(a, s);
 }
 
 }  // namespace
@@ -172,7 +216,7 @@ bool encode_pruned_applicable(const EncodeArgs &a) {
 }
 
 cudaError_t launch_encode_pruned(const EncodeArgs &a, cudaStream_t s) {
-  return (a.rot.wt == QAMW_BF16) ? launch_t<QAMW_BF16>(a, s) : launch_t<QAMW_F32>(a, s);
+  return (a.rot.wt == QAMW_BF16) ? launch_wt<QAMW_BF16>(a, s) : launch_wt<QAMW_F32>(a, s);
 }
 
 }  // namespace qamw

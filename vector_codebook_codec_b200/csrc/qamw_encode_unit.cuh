@@ -10,14 +10,15 @@
 // first (step 5), then bit packing.
 //
 // Work decomposition. A *unit* is one row x 512 consecutive columns handled by
-// one warp: lane l owns columns [16l, 16l + 16) of the unit (8 pairs); the
-// rotation is the fp64 one of qamw_rotate16.cuh, which gives the same x bit
-// for bit as the 1024-column kernel of qamw_encode.cu. A CTA of 28 warps takes
+// one warp with the rotation of qamw_rotate16.cuh (the same x, bit for bit,
+// as the 1024-column kernel of qamw_encode.cu). A CTA of kEncWarps warps takes
 // a contiguous range of *tiles* (one row per warp x one 512-column chunk) in
-// chunk-major order; the chunk's d_j * s_j and 1 / sigma_k live once per CTA in
-// shared memory. The next unit's weights are loaded while the current one is
-// quantized. The search policy S maps the 8 pairs (x0[p], x1[p]) of a lane to
-// 8 indices: S.search8(x0, x1, idx).
+// chunk-major order; the chunk's d_j * s_j and 1 / sigma_k live once per CTA
+// in shared memory. The next unit's weights are loaded while the current one
+// is quantized. After the rotation lane l' holds the unit's pairs
+// 64 (l' >> 3) + 8 m + (l' & 7), m = 0..7; the search policy S maps them to 8
+// indices: S.search8(x0, x1, idx). The indices are staged in the warp's
+// transpose buffer and packed into whole words of the stream.
 #pragma once
 
 #include <cfloat>
@@ -29,27 +30,70 @@
 
 namespace qamw {
 
-constexpr int kUnitWarps = 28;  // warps per CTA = rows per tile; 4096^2 encode: 16 warps 146 us, 20 137, 24 132, 28 126
-constexpr int kUnitThreads = kUnitWarps * 32;
+#ifndef QAMW_ENC_WARPS
+#define QAMW_ENC_WARPS 16
+#endif
+constexpr int kEncWarps = QAMW_ENC_WARPS;   // warps per CTA (one tile row each)
+constexpr int kEncThreads = kEncWarps * 32;
 
 struct ChunkTables {
-  double sd[32 * kSdPitch];         // d_j * s_j of the lane's 16 columns (0 past K)
-  double inv_sigma[32 * kIsPitch];  // 1 / sigma_k of the lane's 8 pairs (0 past K/2)
+  double sd[32 * kSdPitch];         // d_j * s_j of the lane's 16 columns, load layout (0 past K)
+  double inv_sigma[32 * kIsPitch];  // 1 / sigma_k of the lane's 8 pairs, pair layout (0 past K/2)
 };
-constexpr int kStageBytes = 512;    // per warp: 256 uint16 indices of the unit
 // shared memory the pipeline uses at the start of the dynamic area
-constexpr size_t kUnitSmemBytes = sizeof(ChunkTables) + (size_t)kUnitWarps * kStageBytes;
+constexpr size_t kUnitSmemBytes = sizeof(ChunkTables) + (size_t)kEncWarps * kXbufHalf * sizeof(double);
 
-template <int WT, class Search>
+// Packs the unit's np staged indices (stage[k] = index of unit pair k, 0
+// for k >= np) into its words dst[0 .. ceil(np B / 32)). BB > 0 fixes the
+// code size B at compile time (constant divisions and shifts, no inner loop).
+template <int BB>
+__device__ __forceinline__ void pack_unit(const uint16_t *stage, uint32_t *dst, int np, int B, uint64_t divB,
+                                          int lane) {
+  const int nw = (np * B + 31) >> 5;
+  if (BB > 0) {
+    constexpr int kB = BB > 0 ? BB : 1;
+    constexpr int kMore = (32 + kB - 1) / kB;   // indices after the first that can start inside a word
+    for (int w = lane; w < nw; w += 32) {
+      const int bit0 = w * 32;
+      const int k0 = bit0 / kB;
+      const int off0 = k0 * kB - bit0;          // in (-B, 0]
+      uint32_t word = (uint32_t)stage[k0] >> (-off0);
+#pragma unroll
+      for (int i = 1; i <= kMore; ++i) {
+        const int off = off0 + i * kB;          // > 0
+        if (off < 32) word |= (uint32_t)stage[k0 + i] << off;
+      }
+      dst[w] = word;
+    }
+  } else {
+    for (int w = lane; w < nw; w += 32) {
+      const int bit0 = w * 32;
+      const int k0 = (int)(((uint64_t)bit0 * divB) >> 32);               // bit0 / B
+      const int k1 = min((int)(((uint64_t)(bit0 + 31) * divB) >> 32), np - 1);
+      uint32_t word = 0;
+#pragma unroll 1   // 2 to 4 indices per word
+      for (int k = k0; k <= k1; ++k) {
+        const int off = k * B - bit0;
+        const uint32_t iv = stage[k];
+        word |= (off >= 0) ? (iv << off) : (iv >> (-off));
+      }
+      dst[w] = word;
+    }
+  }
+}
+
+// LB > 0 fixes log2 b, BB > 0 the code size, at compile time (0: read at run time).
+template <int WT, int LB, int BB, class Search>
 __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, unsigned char *smem,
                                              const Search &S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const RotateArgs &ra = a.rot;
   ChunkTables &ct = *reinterpret_cast<ChunkTables *>(smem);
-  uint16_t *stage = reinterpret_cast<uint16_t *>(smem + sizeof(ChunkTables) + warp * kStageBytes);
+  double *xbuf = reinterpret_cast<double *>(smem + sizeof(ChunkTables)) + warp * kXbufHalf;
+  uint16_t *stage = reinterpret_cast<uint16_t *>(xbuf);
   const int64_t M = ra.M, K = ra.K, P = K >> 1;
   const int64_t n_chunks = (K + kUnit - 1) / kUnit;
-  const int64_t RG = (M + kUnitWarps - 1) / kUnitWarps;
+  const int64_t RG = (M + kEncWarps - 1) / kEncWarps;
   const int64_t T = n_chunks * RG;
   const int64_t t0 = (int64_t)blockIdx.x * T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
   const double inv_sqrt_b = 1.0 / sqrt((double)(1 << ra.log2b));
@@ -60,7 +104,7 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
 
   // the next unit's weights and row norm, loaded while the current one is searched
   auto prefetch = [&](int64_t chunk, int64_t g, WRegs<WT> &w, float &rn) -> bool {
-    const int64_t row = g * kUnitWarps + warp;
+    const int64_t row = g * kEncWarps + warp;
     rn = 0.0f;
     if (row >= M) return false;
     rn = ra.r[row];
@@ -84,10 +128,10 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
         // a rotated unit row has |y_j| <= 1 (to within the fp32 rounding of r),
         // so |x| <= 1 / sigma_k: every x of the column is a finite fp32 when
         // 1 / sigma_k is at most half the fp32 range (else the status says so)
-        const int i = threadIdx.x;
-        const int64_t p = chunk * (kUnit / 2) + i;
+        const int k = threadIdx.x;
+        const int64_t p = chunk * (kUnit / 2) + k;
         const double is = (p < P) ? 1.0 / (double)a.sigma[p] : 0.0;
-        ct.inv_sigma[(i >> 3) * kIsPitch + (i & 7)] = is;
+        ct.inv_sigma[pair_slot(k)] = is;
         if (!(fabs(is) <= 0.5 * (double)FLT_MAX)) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
       }
       __syncthreads();
@@ -98,60 +142,50 @@ __device__ __forceinline__ void encode_units(const EncodeArgs &a, int vec_ok, un
     const float r = rn_next;
     if (t + 1 < t1) full_next = prefetch(next_chunk, next_g, wn, rn_next);
 
-    const int64_t row = g * kUnitWarps + warp;
+    const int64_t row = g * kEncWarps + warp;
     if (row >= M) continue;
     const int64_t col = chunk * kUnit + 16 * lane;
 
     float x0[8], x1[8];
-    uint32_t bad = 0;
-    if (r > 0.0f && isfinite(r)) {
-      double v[16];
-      scaled16<WT>(v, wc, full, ra.W, ra.ldw, K, row, col, &ct.sd[lane * kSdPitch]);
-      fwht16_fp64(v, ra.log2b, lane);
+    const bool ok = r > 0.0f && isfinite(r);   // uniform across the warp (one row)
+    if (ok) {
+      double u[16];
+      rotate_unit16<WT, true, LB>(u, wc, full, ra.W, ra.ldw, K, row, col, &ct.sd[lane * kSdPitch], ra.log2b,
+                                  xbuf, lane);
       const double qn = inv_sqrt_b / (double)r;
       const double2 *is2 = reinterpret_cast<const double2 *>(&ct.inv_sigma[lane * kIsPitch]);
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const double2 is = is2[h];
         const double f0 = qn * is.x, f1 = qn * is.y;
-        x0[2 * h] = (float)(v[4 * h] * f0);
-        x1[2 * h] = (float)(v[4 * h + 1] * f0);
-        x0[2 * h + 1] = (float)(v[4 * h + 2] * f1);
-        x1[2 * h + 1] = (float)(v[4 * h + 3] * f1);
+        x0[2 * h] = (float)(u[4 * h] * f0);
+        x1[2 * h] = (float)(u[4 * h + 1] * f0);
+        x0[2 * h + 1] = (float)(u[4 * h + 2] * f1);
+        x1[2 * h + 1] = (float)(u[4 * h + 3] * f1);
       }
     } else {
-      if (!(r == 0.0f)) bad = 1;   // NaN / Inf row norm; a zero row codes every pair as x = 0
+      // NaN / Inf row norm: status; a zero row codes every pair as x = 0
+      if (!(r == 0.0f) && lane == 0) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
 #pragma unroll
       for (int p = 0; p < 8; ++p) { x0[p] = 0.0f; x1[p] = 0.0f; }
     }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) status_or(a.status, QAMW_STATUS_NONFINITE_INPUT);
 
     int idx[8];
     S.search8(x0, x1, idx);
 
-    // pack: stage the unit's 256 indices, then build the unit's words
-    __syncwarp();
-    reinterpret_cast<uint4 *>(stage)[lane] =
-        make_uint4((uint32_t)idx[0] | ((uint32_t)idx[1] << 16), (uint32_t)idx[2] | ((uint32_t)idx[3] << 16),
-                   (uint32_t)idx[4] | ((uint32_t)idx[5] << 16), (uint32_t)idx[6] | ((uint32_t)idx[7] << 16));
-    __syncwarp();
+    // pack: stage the unit's 256 indices (in pair order; 0 past the last pair),
+    // then build the unit's words
     const int64_t pair0 = chunk * (kUnit / 2);
     const int np = (int)((P - pair0) < (kUnit / 2) ? (P - pair0) : (kUnit / 2));
-    const int nw = (np * B + 31) >> 5;
-    uint32_t *dst = a.packed + row * a.wpr + chunk * (int64_t)(8 * B);
-    for (int w = lane; w < nw; w += 32) {
-      const int bit0 = w * 32;
-      const int k0 = (int)(((uint64_t)bit0 * divB) >> 32);               // bit0 / B
-      const int k1 = min((int)(((uint64_t)(bit0 + 31) * divB) >> 32), np - 1);
-      uint32_t word = 0;
-#pragma unroll 1   // 2 to 4 indices per word: unrolling measured slower
-      for (int k = k0; k <= k1; ++k) {
-        const int off = k * B - bit0;
-        const uint32_t iv = stage[k];
-        word |= (off >= 0) ? (iv << off) : (iv >> (-off));
-      }
-      dst[w] = word;
+    __syncwarp();   // the transpose buffer is free again
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int k = unit_pair(lane, m);
+      stage[k] = (uint16_t)(k < np ? idx[m] : 0);
     }
+    __syncwarp();
+    pack_unit<BB>(stage, a.packed + row * a.wpr + chunk * (int64_t)(8 * B), np, B, divB, lane);
+    __syncwarp();   // the stage is read before the next unit's transpose overwrites it
   }
 }
 

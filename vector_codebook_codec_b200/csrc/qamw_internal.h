@@ -17,21 +17,53 @@ constexpr int kCalibRowGroup = 28;
 constexpr int kUnitCols = 1024;
 
 // Header of a search table (see qamw_search.cu).
-constexpr uint32_t kSearchMagic = 0x32574D51u;   // "QMW2": table layout version 2
+constexpr uint32_t kSearchMagic = 0x34574D51u;   // "QMW4": table layout version 4 (8-byte cell records)
+constexpr int kSearchMaxG = 181;                 // the scan kernel's limit (32768 cells)
+constexpr int kSearchInline = 3;                 // candidates held in a cell record
+constexpr int kSearchImageOffset = 64;           // bytes from the table's start to the records
 struct SearchHeader {
   uint32_t magic;
-  int32_t N, G, total;
-  int32_t valid, capacity;
+  int32_t N, G, total;     // total: overflow entries used
+  int32_t valid, capacity; // capacity: overflow entries the table holds
   // The grid is uniform in u = T(x) = x / (a + |x|) on each axis: cell index
   // floor((T(x) + UL) * inv_cw), UL = T(L); it covers [-L, L]^2 in x.
   float a, UL, inv_cw, L;
-  int32_t pad[2];
+  int32_t image_bytes;     // records + overflow, a multiple of 16: the bytes the encode copies
+  int32_t pad;
 };
 static_assert(sizeof(SearchHeader) == 48, "search header is 48 bytes");
+// A cell record: four 16-bit fields e0, e1, e2, meta. meta & 3 = n in 1..3:
+// the cell's list is e0..e(n-1) (ascending; unused fields repeat e0). n = 0:
+// the list is e0, e1, e2 followed by ovf[o + 1 .. o + ovf[o]] (o = meta >> 2,
+// ascending), in the table's overflow array.
+__host__ __device__ __forceinline__ uint64_t search_record(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t meta) {
+  return (uint64_t)e0 | ((uint64_t)e1 << 16) | ((uint64_t)e2 << 32) | ((uint64_t)meta << 48);
+}
 int search_grid(int N);
+
+// The encode's cell of a normalised pair: per axis c = round(T(x) * inv_cw +
+// (G - 1) / 2) with T(x) = x / (a + |x|), which for odd G is floor((T(x) + UL)
+// * inv_cw), the grid of the table; -1 outside the grid (|x| > L on an axis,
+// or a non-finite x). The rounding to an integer is that of one fp32 fma at
+// the magnitude 1.5 * 2^23 (unit spacing), cbias = 1.5 * 2^23 + (G - 1) / 2,
+// and the integer is read from the float's bits: no conversion instruction.
+// Its error in cells (approximate reciprocal, two fp32 roundings) is below
+// 1e-4, inside the 1e-3-cell margin every list is built with.
+constexpr float kCellMagic = 12582912.0f;        // 1.5 * 2^23
+constexpr int kCellMagicBits = 0x4B400000;       // its fp32 bits
+__device__ __forceinline__ int search_cell(float x0, float x1, float a, float inv_cw, float cbias, float L, int G) {
+  const float u0 = __fdividef(x0, __fadd_rn(a, fabsf(x0)));
+  const float u1 = __fdividef(x1, __fadd_rn(a, fabsf(x1)));
+  const int cx = __float_as_int(__fmaf_rn(u0, inv_cw, cbias)) - kCellMagicBits;
+  const int cy = __float_as_int(__fmaf_rn(u1, inv_cw, cbias)) - kCellMagicBits;
+  const bool in = fmaxf(fabsf(x0), fabsf(x1)) <= L && (unsigned)cx < (unsigned)G && (unsigned)cy < (unsigned)G;
+  return in ? cy * G + cx : -1;
+}
 int64_t search_capacity(int N);
 size_t search_table_bytes(int N);
 cudaError_t launch_build_search_table(const float *codebook, int N, void *table, cudaStream_t s);
+// Test hook: the encode's cell of n pairs (float32 [n][2]) for a table (-1 off the grid or for an invalid table).
+cudaError_t launch_search_cells(const float *x, int64_t n, const void *table, int32_t *cell_out, cudaStream_t s);
 
 struct ScaleArgs {
   const float *act_rms;  // [K] or nullptr
@@ -132,6 +164,8 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 bool decode_tma_applicable(const DecodeArgs &a);
 cudaError_t launch_decode_tma(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_rotate_test(const RotateTestArgs &a, cudaStream_t s);
+// The same for b <= 512 with the 512-column rotation of the encode and calibrate kernels.
+cudaError_t launch_rotate_test512(const RotateTestArgs &a, cudaStream_t s);
 
 // Lloyd training of the 2D codebook (qamw_lloyd.cu); points and centroids are
 // fp64 [.][2], 16-byte aligned.

@@ -34,16 +34,23 @@
 // than kListMax is kept whole. Pairs outside the grid, or a table that does
 // not fit, use the brute-force search.
 //
-// The encode computes a pair's cell in fp32 as floor((T(x) + UL) * inv_cw)
-// with UL, inv_cw and a read from the header; its rounding error is below
-// 1e-4 of a cell, and the margin of 1e-3 cells that every cell is enlarged
-// by (in u, then mapped back to x in fp64) covers it.
+// The encode computes a pair's cell in fp32 as round(T(x) * inv_cw + (G-1)/2),
+// which for odd G is floor((T(x) + UL) * inv_cw), with inv_cw, a and L read
+// from the header (search_cell in qamw_internal.h); its error is below 1e-4
+// of a cell, and the margin of 1e-3 cells that every cell is enlarged by (in
+// u, then mapped back to x in fp64) covers it.
 //
 // Table layout (device memory owned by the caller, 16-byte aligned):
-//   SearchHeader | uint32 offsets[G*G + 1] | uint16 cand[capacity]
-// cand[offsets[k] .. offsets[k+1]) are the centroid indices of cell
-// k = iy * G + ix in ascending order. The build is four kernels with a fixed
-// order of every reduction, so the table is a pure function of the codebook.
+//   SearchHeader (48 bytes, padded to 64) | uint64 rec[G*G] | uint16 ovf[capacity]
+// rec[k] is the record of cell k = iy * G + ix (qamw_internal.h): up to three
+// candidates inline, longer lists continue in ovf. The records and the
+// overflow array form one image of image_bytes that the encode copies to
+// shared memory with one bulk asynchronous copy. Short lists (one to three
+// entries, ~96% of the pairs on the shipped N = 2048 codebook at G = 137)
+// need no list load at all: the record holds them. The build is four kernels
+// with a fixed order of every reduction, so the table is a pure function of
+// the codebook.
+#include <algorithm>
 #include <cfloat>
 #include <cmath>
 
@@ -54,18 +61,28 @@ namespace qamw {
 
 // The finest grid whose table fits the encode's shared memory with 16-bit
 // offsets (lists + identity list < 65536 entries) for the shipped codebooks.
-int search_grid(int N) { return N >= 2048 ? 176 : (N >= 64 ? 160 : 32); }
+// G is odd, so that the encode finds a cell by rounding (search_cell); the
+// records (8 G^2 bytes) and overflow lists fit the encode's shared memory
+// beside its 16 warps' buffers and the codebook.
+#ifndef QAMW_GRID_LARGE
+#define QAMW_GRID_LARGE 137
+#endif
+#ifndef QAMW_GRID_MID
+#define QAMW_GRID_MID 145
+#endif
+int search_grid(int N) { return N >= 2048 ? QAMW_GRID_LARGE : (N >= 64 ? QAMW_GRID_MID : 33); }
 
-int64_t search_capacity(int N) {
+// Overflow entries (counts included) the table holds: 12288 for N >= 2048,
+// 4096 for smaller codebooks (whose cells hold fewer centroids); sized so
+// that records and overflow fit the encode's shared memory.
+int64_t search_capacity(int N) { return N >= 2048 ? 12288 : 4096; }
+
+static size_t image_bytes(int N) {
   const int G = search_grid(N);
-  return (int64_t)G * G * (N < 64 ? N : 64);   // a cell lists at most N (and in practice far fewer than 64)
+  return ((size_t)G * G * 8 + (size_t)search_capacity(N) * 2 + 15) & ~size_t(15);
 }
 
-size_t search_table_bytes(int N) {
-  const int G = search_grid(N);
-  const size_t off = sizeof(SearchHeader) + (size_t)(G * G + 1) * 4;
-  return (off + (size_t)search_capacity(N) * 2 + 15) & ~size_t(15);
-}
+size_t search_table_bytes(int N) { return (size_t)kSearchImageOffset + image_bytes(N); }
 
 namespace {
 
@@ -95,7 +112,8 @@ __global__ void table_header_kernel(const float *codebook, int N, int G, int64_t
     h->UL = UL;
     h->inv_cw = (float)G / (2.0f * UL);
     h->L = L;
-    h->pad[0] = h->pad[1] = 0;
+    h->image_bytes = 0;
+    h->pad = 0;
     h->valid = 0;
     h->capacity = (int32_t)capacity;
   }
@@ -178,8 +196,9 @@ __device__ bool beaten(const float *codebook, const uint16_t *buf, int n, int k,
   return false;
 }
 
+// Per-cell list length (after pruning) into the record slot, as scratch.
 __global__ void __launch_bounds__(kListThreads) table_count_kernel(const float *codebook, SearchHeader *h,
-                                                                   uint32_t *offsets) {
+                                                                   uint64_t *rec) {
   __shared__ uint16_t bufs[kListThreads / 32][kListMax];
   const int lane = threadIdx.x & 31;
   uint16_t *buf = bufs[threadIdx.x >> 5];
@@ -195,15 +214,16 @@ __global__ void __launch_bounds__(kListThreads) table_count_kernel(const float *
     for (int k = lane; k < n; k += 32) cnt += beaten(codebook, buf, n, k, x0, x1, y0, y1) ? 0 : 1;
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
   }
-  if (lane == 0) offsets[cell + 1] = (uint32_t)cnt;
+  if (lane == 0) rec[cell] = (uint64_t)(uint32_t)cnt;
 }
 
-// Prefix sum of the G*G counts held in offsets[1..n] (one CTA of 1024
-// threads, fixed order). Each thread owns up to kScanPer consecutive cells:
-// it keeps their counts in registers and writes only their offsets, so no
-// slot is read by one thread and written by another.
-constexpr int kScanPer = 32;   // up to 32768 cells (G <= 181) / 1024 threads
-__global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint32_t *offsets) {
+// Overflow offsets: a cell of count c > kSearchInline takes 1 + c - 3
+// overflow entries (its extra count, then its entries beyond the third).
+// Prefix sum in a fixed order (one CTA of 1024 threads); each thread owns up
+// to kScanPer consecutive cells and writes rec[cell] = count | offset << 32.
+constexpr int kScanPer = 32;   // up to 32768 cells (G <= kSearchMaxG) / 1024 threads
+__device__ __forceinline__ uint32_t ovf_size(uint32_t c) { return c > (uint32_t)kSearchInline ? c - kSearchInline + 1 : 0u; }
+__global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint64_t *rec) {
   __shared__ uint32_t wsum[32];
   const int n = h->G * h->G;
   const int b = threadIdx.x * kScanPer;
@@ -211,8 +231,8 @@ __global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint3
   uint32_t s = 0;
 #pragma unroll
   for (int k = 0; k < kScanPer; ++k) {
-    cnt[k] = (b + k < n) ? offsets[b + k + 1] : 0u;
-    s += cnt[k];
+    cnt[k] = (b + k < n) ? (uint32_t)rec[b + k] : 0u;
+    s += ovf_size(cnt[k]);
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t inc = s;
@@ -231,39 +251,49 @@ __global__ void __launch_bounds__(1024) table_scan_kernel(SearchHeader *h, uint3
     wsum[lane] = w;
   }
   __syncthreads();
-  uint32_t run = inc - s + (warp > 0 ? wsum[warp - 1] : 0u);
+  uint32_t run = inc - s + (warp > 0 ? wsum[warp - 1] : 0u);   // overflow entries before this thread's cells
 #pragma unroll
   for (int k = 0; k < kScanPer; ++k) {
     if (b + k < n) {
-      run += cnt[k];
-      offsets[b + k + 1] = run;
+      rec[b + k] = (uint64_t)cnt[k] | ((uint64_t)run << 32);
+      run += ovf_size(cnt[k]);
     }
   }
-  if (threadIdx.x == 0) offsets[0] = 0u;
   if (b < n && b + kScanPer >= n) {   // the thread that owns the last cell
     h->total = (int32_t)run;
-    h->valid = ((int64_t)run <= (int64_t)h->capacity) ? 1 : 0;
+    // offsets are 14-bit fields of the records
+    h->valid = ((int64_t)run <= (int64_t)h->capacity && run < (1u << 14)) ? 1 : 0;
+    h->image_bytes = (int32_t)(((size_t)n * 8 + (size_t)h->capacity * 2 + 15) & ~size_t(15));
   }
 }
 
+// The final records and overflow lists. The warp writes its list's entries by
+// position: positions 0..2 into the record, later ones into the overflow.
 __global__ void __launch_bounds__(kListThreads) table_fill_kernel(const float *codebook, const SearchHeader *h,
-                                                                  const uint32_t *offsets, uint16_t *cand) {
+                                                                  uint64_t *rec, uint16_t *ovf) {
   __shared__ uint16_t bufs[kListThreads / 32][kListMax];
-  const int lane = threadIdx.x & 31;
-  uint16_t *buf = bufs[threadIdx.x >> 5];
+  __shared__ uint32_t heads[kListThreads / 32][kSearchInline];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  uint16_t *buf = bufs[wib];
   const int cell = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
   const SearchHeader hh = *h;
   if (!hh.valid || cell >= hh.G * hh.G) return;
+  const uint64_t scratch = rec[cell];
+  const uint32_t count = (uint32_t)scratch, off = (uint32_t)(scratch >> 32);
   double x0, x1, y0, y1;
   cell_bounds(hh, cell, x0, x1, y0, y1);
   const int n = first_test(codebook, hh.N, x0, x1, y0, y1, lane, buf);
-  uint32_t pos = offsets[cell];
+  auto emit = [&](uint32_t pos, uint32_t idx) {
+    if (pos < (uint32_t)kSearchInline) heads[wib][pos] = idx;
+    else ovf[off + 1 + (pos - kSearchInline)] = (uint16_t)idx;
+  };
+  uint32_t pos = 0;
   if (n <= kListMax) {
     for (int base = 0; base < n; base += 32) {
       const int k = base + lane;
       const bool keep = k < n && !beaten(codebook, buf, n, k, x0, x1, y0, y1);
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) cand[pos + __popc(m & ((1u << lane) - 1u))] = buf[k];
+      if (keep) emit(pos + __popc(m & ((1u << lane) - 1u)), buf[k]);
       pos += __popc(m);
     }
   } else {   // too long to prune: the whole first-test list
@@ -272,30 +302,58 @@ __global__ void __launch_bounds__(kListThreads) table_fill_kernel(const float *c
       const int i = base + lane;
       const bool keep = i < hh.N && dmin2(codebook[2 * i], codebook[2 * i + 1], x0, x1, y0, y1) <= bound;
       const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) cand[pos + __popc(m & ((1u << lane) - 1u))] = (uint16_t)i;
+      if (keep) emit(pos + __popc(m & ((1u << lane) - 1u)), (uint32_t)i);
       pos += __popc(m);
     }
   }
+  __syncwarp();
+  if (lane == 0) {
+    // pos == count: both passes see the same lists
+    const uint32_t e0 = heads[wib][0];
+    const uint32_t e1 = count > 1 ? heads[wib][1] : e0, e2 = count > 2 ? heads[wib][2] : e0;
+    uint32_t meta = count;
+    if (count > (uint32_t)kSearchInline) {
+      ovf[off] = (uint16_t)(count - kSearchInline);
+      meta = off << 2;
+    }
+    rec[cell] = search_record(e0, e1, e2, meta);
+  }
+}
+
+// Test hook: the encode's cell computation on given pairs.
+__global__ void search_cells_kernel(const float *x, int64_t n, const SearchHeader *h, int32_t *cell_out) {
+  const SearchHeader hh = *h;
+  const bool ok = hh.magic == kSearchMagic && hh.valid == 1 && hh.G >= 1 && hh.G <= kSearchMaxG && (hh.G & 1) == 1;
+  const float cbias = kCellMagic + (float)((hh.G - 1) / 2);
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    cell_out[i] = ok ? search_cell(x[2 * i], x[2 * i + 1], hh.a, hh.inv_cw, cbias, hh.L, hh.G) : -1;
 }
 
 }  // namespace
 
+cudaError_t launch_search_cells(const float *x, int64_t n, const void *table, int32_t *cell_out, cudaStream_t s) {
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
+  search_cells_kernel<<<(int)std::max<int64_t>(blocks, 1), 256, 0, s>>>(
+      x, n, reinterpret_cast<const SearchHeader *>(table), cell_out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_build_search_table(const float *codebook, int N, void *table, cudaStream_t s) {
   const int G = search_grid(N);
   SearchHeader *h = reinterpret_cast<SearchHeader *>(table);
-  uint32_t *offsets = reinterpret_cast<uint32_t *>(reinterpret_cast<unsigned char *>(table) + sizeof(SearchHeader));
-  uint16_t *cand = reinterpret_cast<uint16_t *>(offsets + G * G + 1);
+  uint64_t *rec = reinterpret_cast<uint64_t *>(reinterpret_cast<unsigned char *>(table) + kSearchImageOffset);
+  uint16_t *ovf = reinterpret_cast<uint16_t *>(rec + (size_t)G * G);
   table_header_kernel<<<1, 1024, 0, s>>>(codebook, N, G, search_capacity(N), h);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int cells = G * G;
   const int threads = kListThreads;
   const int blocks = (cells * 32 + threads - 1) / threads;
-  table_count_kernel<<<blocks, threads, 0, s>>>(codebook, h, offsets);
+  table_count_kernel<<<blocks, threads, 0, s>>>(codebook, h, rec);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  table_scan_kernel<<<1, 1024, 0, s>>>(h, offsets);
+  table_scan_kernel<<<1, 1024, 0, s>>>(h, rec);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  table_fill_kernel<<<blocks, threads, 0, s>>>(codebook, h, offsets, cand);
+  table_fill_kernel<<<blocks, threads, 0, s>>>(codebook, h, rec, ovf);
   return cudaGetLastError();
 }
 
