@@ -42,11 +42,11 @@ FALLBACK_HBM_GBS = 6650.0
 SM_COUNT_B200 = 148
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + written) of one encode_pruned_kernel launch, from the ncu
-# capture in profiles/encode_pruned_kernel_4096x4096_bf16_N2048.md (default
-# workload only). Valid while that kernel is unchanged; set to None after a
-# change until it is captured again.
-ENCODE_TRAFFIC_BYTES = {"llama7b_attn": 34437120 + 123648}
+# DRAM bytes (read + written) of one launch of the encode kernel on a
+# workload, from one ncu capture of that kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum); an entry is removed whenever the kernel changes,
+# until it is captured again.
+ENCODE_TRAFFIC_BYTES = {}
 
 
 def parse_args(argv=None):
@@ -56,12 +56,15 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="llama7b_attn",
-                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4", "lloyd", "polar"),
+                   choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4", "lloyd", "polar", "mlp",
+                            "stack_1p1b"),
                    help="llama7b_attn: 4096x4096 bf16 at 2048 centroids (5.5 bits/weight; the default); "
                         "rate35 / rate4: the same matrix at 128 / 256 centroids (3.5 / 4 bits/weight); "
                         "decode_13b: decode-only sweep over the 13B shapes; tiny: 256x512 fp32; "
                         "lloyd: codebook training, one Lloyd iteration of 2048 centroids on 2^21 samples per step; "
-                        "polar: the polar baseline codec on the 4096x4096 projection at 2048 points")
+                        "polar: the polar baseline codec on the 4096x4096 projection at 2048 points; "
+                        "mlp: the 24 MLP runs (11008x4096 and 4096x11008, alpha x block x codebook); "
+                        "stack_1p1b: the 154 matrices of the 22-layer 1.1B-shaped stack")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
@@ -187,23 +190,87 @@ def oracle_sample_step(W32_rows, act, spec, C):
     codec.decode(enc["packed"], enc["r"], sig, act, spec.alpha, spec.K, spec.block, spec.seed, C, spec.bits)
 
 
-def time_oracle(W32, act, spec, C, rows, repeats):
+_WORKER_LIMITS = None
+
+
+def _oracle_worker_init():
+    """Each oracle worker process runs numpy on one thread (the pool supplies the parallelism)."""
+    global _WORKER_LIMITS
     from threadpoolctl import threadpool_limits
-    sample = W32[:rows]
-    times = []
-    with threadpool_limits(limits=1):
-        for _ in range(repeats):
-            t0 = time.perf_counter()
-            oracle_sample_step(sample, act, spec, C)
-            times.append(time.perf_counter() - t0)
-    return times
+    _WORKER_LIMITS = threadpool_limits(limits=1)
+
+
+def _oracle_task(job):
+    W_rows, act, spec, C = job
+    oracle_sample_step(W_rows, act, spec, C)
+    return W_rows.shape[0]
+
+
+class OraclePool:
+    """The oracle on every host core: a pool of spawned worker processes (one
+    numpy thread each), each running the whole calibrate + encode + decode
+    of its own block of rows. Spawned, not forked, so that it is safe next to
+    a CUDA context."""
+
+    def __init__(self, workers=None):
+        import multiprocessing as mp
+        self.workers = int(workers or os.cpu_count() or 1)
+        self.pool = mp.get_context("spawn").Pool(self.workers, initializer=_oracle_worker_init)
+
+    def run(self, W32, act, spec, C, rows_per_worker, start=0):
+        """One parallel step over workers x rows_per_worker rows; returns (rows, wall seconds)."""
+        M = W32.shape[0]
+        jobs = []
+        for w in range(self.workers):
+            r0 = (start + w * rows_per_worker) % M
+            idx = (np.arange(rows_per_worker) + r0) % M
+            jobs.append((np.ascontiguousarray(W32[idx]), act, spec, C))
+        t0 = time.perf_counter()
+        rows = sum(self.pool.map(_oracle_task, jobs))
+        return rows, time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def time_oracle_parallel(pool, W32, act, spec, C, rows_per_worker, repeats, warmup=1):
+    for i in range(warmup):
+        pool.run(W32, act, spec, C, rows_per_worker, start=i)
+    walls, rows = [], 0
+    for i in range(repeats):
+        rows, wall = pool.run(W32, act, spec, C, rows_per_worker, start=warmup + i)
+        walls.append(wall)
+    return rows, walls
 
 
 def auto_rows(spec):
-    """Rows per oracle sample: ~4 s of single-core fp64 work (64 rows of the
-    4096-column, N = 2048 workload; the brute-force search dominates)."""
+    """Rows per oracle worker per step: ~1 s of single-core fp64 work (16 rows
+    of the 4096-column, N = 2048 workload; the brute-force search dominates)."""
     per_row = spec.K / 2 * spec.N
-    return max(1, min(spec.M, int(round(64 * 2048 * 2048 / per_row))))
+    return max(1, min(spec.M, int(round(16 * 2048 * 2048 / per_row))))
+
+
+def oracle_parity(W32, act, spec, C, sigma, r, s, packed):
+    """Index parity of the whole matrix (every pair): the oracle's fp64
+    rotation, sigma and exact nearest centroids (oracle.codec.nearest_centroid_kd)
+    against the GPU's packed stream, sigma, row norms and channel scales."""
+    from oracle import codec
+    t0 = time.perf_counter()
+    s_o, r_o, Y = codec.rotated_rows(W32, act, spec.alpha, spec.block, spec.seed)
+    sig_o = codec.sigma_from_rotated(Y)
+    X = codec.normalised_pairs(Y, sig_o)
+    del Y
+    idx, gap = codec.nearest_centroid_kd(X, C)
+    gidx = codec.unpack_indices(packed, spec.K // 2, spec.bits)
+    diff = gidx != idx
+    near = diff & (gap < 1e-6)
+    return {"scope": f"every pair of the {spec.M}x{spec.K} matrix", "pairs": int(idx.size),
+            "near_tie_pairs": int(np.sum(gap < 1e-6)), "hard_mismatches": int(np.sum(diff & ~near)),
+            "near_tie_mismatches": int(np.sum(near)), "sigma_mismatches": int(np.sum(sigma != sig_o)),
+            "row_norm_mismatches": int(np.sum(r != r_o)), "scale_mismatches": int(np.sum(s != s_o)),
+            "rule": "indices bit-exact unless the oracle's best-two gap is below 1e-6 (counted); sigma, r, s bit-exact",
+            "oracle_seconds": round(time.perf_counter() - t0, 1)}
 
 
 def _reference_line(args, metric, value, unit, config, sample, ms_per_step, cores=1):
@@ -299,19 +366,24 @@ def run_reference(args):
     act = synth.act_for(spec)
     C = q.load_codebook(spec.N)
     rows = args.cpu_rows or auto_rows(spec)
-    for _ in range(args.warmup):
-        time_oracle(W32, act, spec, C, rows, 1)
-    times = time_oracle(W32, act, spec, C, rows, args.steps)
-    tot = sum(times)
-    value = rows * spec.K * args.steps / tot / 1e9
+    pool = OraclePool()
+    try:
+        nrows, walls = time_oracle_parallel(pool, W32, act, spec, C, rows, args.steps, warmup=max(1, args.warmup))
+    finally:
+        pool.close()
+    tot = sum(walls)
+    value = nrows * spec.K * args.steps / tot / 1e9
+    sample = (f"{pool.workers} worker processes x {rows} rows (of {spec.M}) per step, each running calibrate + "
+              f"encode + decode of its rows on one core" + (f"; {spec.name}, the first matrix of the workload"
+                                                             if args.workload in ("mlp", "stack_1p1b") else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wname, "M": spec.M, "K": spec.K, "block": spec.block, "N": spec.N,
                    "bits": spec.bits, "alpha": spec.alpha, "weight_dtype": spec.dtype},
-        "cpu_baseline": {"value": value, "unit": "Gweights/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {rows} of {spec.M} rows per step (calibrate + encode + decode)"},
+        "cpu_baseline": {"value": value, "unit": "Gweights/s", "cores": pool.workers, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "Gweights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -323,18 +395,20 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 
 def pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec) -> int:
-    """Distance evaluations the exact pruned search performs on this matrix: for
-    every pair, the length of its grid cell's candidate list, or N for a pair
+    """Distance evaluations the exact pruned search performs on this matrix:
+    three per pair (the inline entries of its cell's record, evaluated without
+    a branch), plus the overflow entries of a longer list, or N for a pair
     outside the grid. x is recomputed through the library's fp64 rotation hook
-    (qamw_rotate_rows) on U = w * s / r, in row blocks; the cell arithmetic is
-    the encode's fp32 one, on the table header's constants."""
+    (qamw_rotate_rows) on U = w * s / r, in row blocks, and each pair's cell
+    comes from the encode's own cell arithmetic (qamw_search_cells)."""
     import torch
-    raw = table[:48].cpu().numpy()
+    raw = table.cpu().numpy()
     G = int(raw[8:12].view(np.int32)[0])
-    a, UL, inv = (float(v) for v in raw[24:36].view(np.float32))
-    nbytes_off = 4 * (G * G + 1)
-    offsets = table[48:48 + nbytes_off].view(torch.int32).to(torch.int64)
-    lens = (offsets[1:] - offsets[:-1])
+    rec = raw[64:64 + 8 * G * G].view(np.uint64)
+    ovf = raw[64 + 8 * G * G:].view(np.uint16).astype(np.int64)
+    meta = (rec >> np.uint64(48)).astype(np.int64)
+    extra = np.where((meta & 3) == 0, ovf[np.minimum(meta >> 2, ovf.size - 1)], 0)
+    extra_t = torch.from_numpy(extra).to(Wd.device)
     M, K = Wd.shape
     sig = sigma.to(torch.float64)
     total = 0
@@ -344,12 +418,9 @@ def pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec) -> int:
         rr = rnorm[r0:r1].to(torch.float64)[:, None]
         U = torch.where(rr > 0, U / torch.where(rr > 0, rr, torch.ones_like(rr)), torch.zeros_like(U))
         Y = q.rotate_rows(U.contiguous(), spec.block, spec.seed)
-        x = (Y.view(r1 - r0, K // 2, 2) / sig[None, :, None]).to(torch.float32)
-        u = x / (a + x.abs())
-        f = (u + UL) * inv
-        inside = (f >= 0).all(-1) & (f < G).all(-1)
-        cell = f[..., 1].clamp(0, G - 1).to(torch.int64) * G + f[..., 0].clamp(0, G - 1).to(torch.int64)
-        n = torch.where(inside, lens[cell], torch.full_like(cell, spec.N))
+        x = (Y.view(-1, 2) / sig.repeat(r1 - r0)[:, None]).to(torch.float32).contiguous()
+        cells = q.search_cells(x, table).to(torch.int64)
+        n = 3 + torch.where(cells >= 0, extra_t[cells.clamp(min=0)], torch.full_like(cells, spec.N))
         total += int(n.sum().item())
     return total
 
@@ -677,7 +748,259 @@ def run_polar(args):
     return 0
 
 
+def run_multi(args):
+    """Steps over every matrix of a multi-matrix workload: the 24 MLP runs
+    (11008x4096 and 4096x11008 Student-t matrices x alpha {0.25, 0.5, 0.75} x
+    block {128, 256} x {1024, 2048} centroids) or the 154 matrices of the
+    22-layer 1.1B-shaped stack. One step = qamw_calibrate_encode of every
+    matrix, then qamw_decode (bf16) of every matrix, all through the C ABI.
+    Matrices are spread over 4 streams so that small ones (the 256x2048 k and v
+    projections) run beside others. The step is captured once as a CUDA graph
+    and replayed (the headline); per-shape times come from an eager pass with
+    one stream."""
+    import torch
+    import synth
+    import vector_codebook_codec_b200 as q
+    from vector_codebook_codec_b200 import build as qbuild
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    qbuild.build()
+    lib = q.load_library()
+    wl = synth.mlp_runs() if args.workload == "mlp" else synth.stack_1p1b()
+    specs = wl.specs
+    n_streams = 4
+    cache, host_w, ents = {}, {}, []
+    cbs, tables = {}, {}
+    for spec in specs:
+        key = (spec.M, spec.K, spec.dist, spec.std, spec.outlier_frac, spec.outlier_scale, spec.seed)
+        if key not in cache:
+            Wt, _ = synth.to_bf16(synth.make_matrix(spec))
+            cache[key] = Wt.to(dev)
+            host_w[key] = Wt
+        if spec.N not in cbs:
+            cbs[spec.N] = torch.from_numpy(q.load_codebook(spec.N)).to(dev)
+            tables[spec.N] = q.build_search_table(cbs[spec.N])
+        M, K = spec.M, spec.K
+        wpr = q.words_per_row(K, spec.bits)
+        ents.append(dict(
+            spec=spec, key=key, W=cache[key], act=torch.from_numpy(synth.act_for(spec)).to(dev),
+            ws=torch.empty(int(lib.qamw_calibrate_workspace_bytes(M, K)), dtype=torch.uint8, device=dev),
+            sigma=torch.empty(K // 2, dtype=torch.float32, device=dev),
+            packed=torch.empty((M, wpr), dtype=torch.int32, device=dev),
+            r=torch.empty(M, dtype=torch.float32, device=dev), s=torch.empty(K, dtype=torch.float32, device=dev),
+            out=torch.empty((M, K), dtype=torch.bfloat16, device=dev)))
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    main = torch.cuda.current_stream(dev)
+    streams = [torch.cuda.Stream(dev) for _ in range(n_streams)]
+
+    def enc_call(e, st):
+        sp = e["spec"]
+        return q.calibrate_encode(e["W"], e["act"], sp.alpha, sp.block, sp.seed, cbs[sp.N], sp.bits, status=status,
+                                  out=(e["packed"], e["r"], e["s"], e["sigma"]), search_table=tables[sp.N],
+                                  workspace=e["ws"], stream=st)
+
+    def dec_call(e, enc, st):
+        q.decode(enc, cbs[e["spec"].N], out_dtype=torch.bfloat16, status=status, out=e["out"], stream=st)
+
+    def step(origin):
+        """All encodes, then all decodes, round-robin over the streams, forked from and joined to origin."""
+        fork = torch.cuda.Event()
+        fork.record(origin)
+        for st in streams:
+            st.wait_event(fork)
+        encs = [enc_call(e, streams[i % n_streams]) for i, e in enumerate(ents)]
+        for i, (e, enc) in enumerate(zip(ents, encs)):
+            dec_call(e, enc, streams[i % n_streams])
+        for st in streams:
+            j = torch.cuda.Event()
+            j.record(st)
+            origin.wait_event(j)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step(main)
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()} after warm-up")
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    with torch.cuda.graph(graph, stream=side):
+        step(side)
+    for _ in range(args.warmup):
+        flush.fill_(3.0)
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    # eager pass on one stream, each call timed: the per-shape figures
+    per = []
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in ents]
+    flush.fill_(4.0)
+    for e, (a, b, c) in zip(ents, evs):
+        a.record(main)
+        enc = enc_call(e, main)
+        b.record(main)
+        dec_call(e, enc, main)
+        c.record(main)
+    torch.cuda.synchronize(dev)
+    for e, (a, b, c) in zip(ents, evs):
+        per.append((e["spec"], a.elapsed_time(b), b.elapsed_time(c)))
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for i, (e0, e1) in enumerate(gev):
+        flush.fill_(float(i))
+        e0.record(main)
+        graph.replay()
+        e1.record(main)
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()} in the timed steps")
+    total_s = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in gev) / 1e3, dev)
+    weights = sum(sp.M * sp.K for sp in specs)
+    value = aggregate_throughput(weights * args.steps, total_s, world) / 1e9
+    mean_step_s = total_s / args.steps
+
+    # per shape (or per run): mean eager time of the fused encode call and the decode
+    groups = {}
+    for sp, te, td in per:
+        name = sp.name.split(".", 1)[1] if args.workload == "stack_1p1b" else sp.name
+        g = groups.setdefault(name, {"M": sp.M, "K": sp.K, "N": sp.N, "block": sp.block, "alpha": sp.alpha,
+                                     "n": 0, "enc_ms": 0.0, "dec_ms": 0.0})
+        g["n"] += 1
+        g["enc_ms"] += te
+        g["dec_ms"] += td
+    per_shape = []
+    for name, g in groups.items():
+        em, dm = g["enc_ms"] / g["n"], g["dec_ms"] / g["n"]
+        w = g["M"] * g["K"]
+        per_shape.append({"name": name, "M": g["M"], "K": g["K"], "N": g["N"], "block": g["block"],
+                          "alpha": g["alpha"], "matrices": g["n"], "calibrate_encode_us": 1e3 * em,
+                          "decode_us": 1e3 * dm, "gweights_per_s": w / ((em + dm) * 1e-3) / 1e9})
+
+    # the dominant kernel alone on the workload's first matrix (as the default line)
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    e = ents[0]
+    sp = e["spec"]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+    for e0, e1 in kev:
+        flush.fill_(5.0)
+        e0.record(main)
+        q.encode_prepared(e["W"], e["s"], e["r"], sp.block, sp.seed, e["sigma"], cbs[sp.N], sp.bits, status=status,
+                          out=e["packed"], search_table=tables[sp.N])
+        e1.record(main)
+    torch.cuda.synchronize(dev)
+    kern_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in kev)
+    wpr = q.words_per_row(sp.K, sp.bits)
+    enc_bytes = sp.M * sp.K * 2 + sp.M * wpr * 4 + 4 * sp.M + 4 * sp.K + 2 * sp.K + 8 * sp.N
+    roof = {"bound": "hbm", "achieved": enc_bytes / (kern_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": enc_bytes / (kern_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+            "kernel": f"encode_pruned_kernel alone (qamw_encode_prepared) on {sp.name} {sp.M}x{sp.K}",
+            "us_per_launch": 1e3 * kern_ms, "algorithmic_bytes_per_launch": enc_bytes,
+            "peak_source": f"{peak_kind} hbm_gbs"}
+
+    # end to end: every distinct matrix uploaded from pinned host memory, every
+    # matrix's decoded weights and encoded artefact read back, inside the timing
+    e2e = None
+    if not args.no_e2e:
+        pin_w = {k: v.pin_memory() for k, v in host_w.items()}
+        pin_out = [torch.empty(e["out"].shape, dtype=torch.bfloat16).pin_memory() for e in ents]
+        pin_pk = [torch.empty(e["packed"].shape, dtype=torch.int32).pin_memory() for e in ents]
+        pin_meta = [[torch.empty(e[k].shape, dtype=torch.float32).pin_memory() for k in ("r", "s", "sigma")]
+                    for e in ents]
+        h2d = sum(v.numel() * 2 for v in pin_w.values())
+        d2h = sum(o.numel() * 2 + p.numel() * 4 + 4 * (e["spec"].M + e["spec"].K + e["spec"].K // 2)
+                  for o, p, e in zip(pin_out, pin_pk, ents))
+
+        def e2e_step():
+            for k, v in pin_w.items():
+                cache[k].copy_(v, non_blocking=True)
+            step(main)
+            for e, o, p, mt in zip(ents, pin_out, pin_pk, pin_meta):
+                o.copy_(e["out"], non_blocking=True)
+                p.copy_(e["packed"], non_blocking=True)
+                for h, k in zip(mt, ("r", "s", "sigma")):
+                    h.copy_(e[k], non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        for _ in range(max(1, args.steps // 2)):
+            e2e_step()
+        e1.record(main)
+        torch.cuda.synchronize(dev)
+        n_e2e = max(1, args.steps // 2)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+        e2e = {"value": aggregate_throughput(weights * n_e2e, e2e_s, world) / 1e9, "unit": "Gweights/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipelining": "none: uploads, the step on 4 streams, then the read-backs"}
+
+    cpu, parity = None, None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sp0 = specs[0]
+        _, W32 = synth.to_bf16(synth.make_matrix(sp0))
+        act0 = synth.act_for(sp0)
+        C0 = q.load_codebook(sp0.N)
+        rows = args.cpu_rows or auto_rows(sp0)
+        pool = OraclePool()
+        try:
+            nrows, walls = time_oracle_parallel(pool, W32, act0, sp0, C0, rows, 3)
+        finally:
+            pool.close()
+        cpu = {"value": nrows * sp0.K / statistics.median(walls) / 1e9, "unit": "Gweights/s",
+               "cores": pool.workers, "kind": "oracle",
+               "sample": f"{sp0.name} ({sp0.M}x{sp0.K}): {pool.workers} worker processes x {rows} rows per step, "
+                         f"calibrate + encode + decode; median of 3 steps"}
+        # whole-matrix parity of the first matrix (the MLP workload) or of
+        # every matrix of layer 0 (the stack), from the last step's encodings
+        chk = [ents[0]] if args.workload == "mlp" else [e for e in ents if e["spec"].name.startswith("L0.")]
+        parity = {"matrices": [], "pairs": 0, "near_tie_pairs": 0, "hard_mismatches": 0, "near_tie_mismatches": 0,
+                  "sigma_mismatches": 0, "row_norm_mismatches": 0, "scale_mismatches": 0}
+        for e in chk:
+            spx = e["spec"]
+            _, Wx = synth.to_bf16(synth.make_matrix(spx))
+            rec = oracle_parity(Wx, synth.act_for(spx), spx, q.load_codebook(spx.N), e["sigma"].cpu().numpy(),
+                                e["r"].cpu().numpy(), e["s"].cpu().numpy(), e["packed"].cpu().numpy().view(np.uint32))
+            parity["matrices"].append(f"{spx.name} {spx.M}x{spx.K}")
+            for k in ("pairs", "near_tie_pairs", "hard_mismatches", "near_tie_mismatches", "sigma_mismatches",
+                      "row_norm_mismatches", "scale_mismatches"):
+                parity[k] += rec[k]
+        parity["rule"] = "indices bit-exact unless the oracle's best-two gap is below 1e-6 (counted); sigma, r, s bit-exact"
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * mean_step_s, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no checkpoint)",
+                "config": {"workload": wl.name, "matrices": len(specs), "weights_per_step": weights,
+                           "weight_dtype": "bf16", "op": "calibrate + encode all, then decode all (bf16 out)",
+                           "streams": n_streams, "l2": "flushed by a 256 MiB write before every timed step",
+                           "parallelism": f"{world} independent replica(s)"},
+                "roofline": roof, "per_shape": per_shape, "cpu_baseline": cpu, "parity": parity, "e2e": e2e,
+                "gpu_launches": 6 * len(specs) * args.steps, "clocks": clk,
+                "timing": "each step replays one CUDA graph of all calls (4 streams); per_shape: an eager pass"}
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def run_ours(args):
+    if args.workload in ("mlp", "stack_1p1b"):
+        return run_multi(args)
     if args.workload == "polar":
         return run_polar(args)
     if args.workload == "decode_13b":
@@ -830,57 +1153,69 @@ def run_ours(args):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     fp32_peak = sms * FP32_LANES_PER_SM * sm_max * 1e6  # FP32 lane-instructions per second
     P = M * K // 2
+    es = 2 if spec.dtype == "bf16" else 4
     enc_ms = statistics.mean(t_enc)
     dec_ms = statistics.mean(t_dec)
     cal_ms = statistics.mean(t_cal)
     dec_bytes = M * K * 2 + M * wpr * 4 + 4 * M + 4 * K + 2 * K + 8 * spec.N
-    cal_bytes = M * K * 2 * 2 + 4 * K + 4 * M
+    cal_bytes = M * K * es * 2 + 4 * K + 4 * M
     fp32_src = f"{sms} SMs x 128 FP32 lanes x {sm_max:.0f} MHz ({peak_kind} max clock)"
+
+    # The dominant kernel alone: the encode kernel, launched by
+    # qamw_encode_prepared with the step's channel scales and row norms (the
+    # same kernel and inputs as inside qamw_calibrate_encode), timed with
+    # events on this stream after the steps, L2 flushed before each launch.
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(max(args.steps, 3))]
+    for e0, e1 in kev:
+        flush.fill_(5.0)
+        e0.record(stream)
+        q.encode_prepared(Wd, cscale, rnorm, spec.block, spec.seed, sigma, Cd, spec.bits, status=status, out=packed,
+                          search_table=table)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    kern_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in kev)
+    enc_bytes = M * K * es + M * wpr * 4 + 4 * M + 4 * K + 4 * (K // 2) + 8 * spec.N
+    evals = pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec) if args.search == "pruned" else P * spec.N
+    enc_roof = {"bound": "hbm", "achieved": enc_bytes / (kern_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": enc_bytes / (kern_ms * 1e-3) / 1e9 / hbm,
+                "traffic": ENCODE_TRAFFIC_BYTES.get(args.workload if args.search == "pruned" else "-"),
+                "kernel": ("encode_pruned_kernel" if args.search == "pruned" else "encode_kernel (brute force)") +
+                          " alone (qamw_encode_prepared)",
+                "us_per_launch": 1e3 * kern_ms, "algorithmic_bytes_per_launch": enc_bytes,
+                "bytes_note": "weights read + packed words written + r, s, sigma and codebook",
+                "peak_source": f"{peak_kind} hbm_gbs",
+                "fp32_issue": {"achieved": 4.0 * evals / (kern_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
+                               "unit": "G lane-op/s", "frac": 4.0 * evals / (kern_ms * 1e-3) / fp32_peak,
+                               "evaluations_per_pair": evals / P, "peak_source": fp32_src,
+                               "note": "4 FP32 lane-ops (2 FSUB, FMUL, FFMA) per distance evaluation"}}
     # brute-force encode, timed on its own (not part of the step): its search is
     # FP32-bound, 4 FP32 operations (2 FSUB, FMUL, FFMA) per pair and centroid
     brute_ms = None
     if args.search == "pruned" and args.brute_steps > 0:
         bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.brute_steps)]
-        q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sigma, Cd, spec.bits, status=status,
-                 out=(packed, rnorm, cscale))
+        bpk = torch.empty_like(packed)
+        q.encode_prepared(Wd, cscale, rnorm, spec.block, spec.seed, sigma, Cd, spec.bits, status=status, out=bpk)
         for e0, e1 in bev:
             flush.fill_(2.0)
             e0.record(stream)
-            q.encode(Wd, actd, spec.alpha, spec.block, spec.seed, sigma, Cd, spec.bits, status=status,
-                     out=(packed, rnorm, cscale))
+            q.encode_prepared(Wd, cscale, rnorm, spec.block, spec.seed, sigma, Cd, spec.bits, status=status,
+                              out=bpk)
             e1.record(stream)
         torch.cuda.synchronize(dev)
         brute_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in bev)
-        # restore the pruned encoding (identical by construction) for e2e / checks
-        one()
-        torch.cuda.synchronize(dev)
+        if not torch.equal(bpk, packed):
+            raise SystemExit("brute-force and pruned encodes differ")
     elif args.search == "brute":
-        brute_ms = enc_ms
+        brute_ms = kern_ms
     brute_roof = None
     if brute_ms is not None:
         ops = 4.0 * P * spec.N
         brute_roof = {"bound": "alu", "achieved": ops / (brute_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
                       "unit": "Gop/s", "frac": ops / (brute_ms * 1e-3) / fp32_peak, "traffic": None,
-                      "kernel": "encode_kernel (brute-force search; events span the qamw_encode call)",
+                      "kernel": "encode_kernel (brute-force search) alone (qamw_encode_prepared, no table)",
                       "ms": brute_ms, "peak_source": fp32_src}
-    if args.search == "pruned":
-        evals = pruned_evaluations(q, Wd, cscale, rnorm, sigma, table, spec)
-        ops = 4.0 * evals
-        enc_roof = {"bound": "alu", "achieved": ops / (enc_ms * 1e-3) / 1e9, "peak": fp32_peak / 1e9,
-                    "unit": "Gop/s", "frac": ops / (enc_ms * 1e-3) / fp32_peak,
-                    "traffic": ENCODE_TRAFFIC_BYTES.get(args.workload),
-                    "traffic_note": "DRAM bytes per encode_pruned_kernel launch from one ncu capture "
-                                    "(profiles/); the algorithmic bytes are the weights read and the "
-                                    "packed words written",
-                    "kernel": "encode_pruned_kernel (exact pruned search; events span the qamw_encode call)",
-                    "evaluations_per_pair": evals / P, "peak_source": fp32_src,
-                    "brute_force_equivalent_frac": 4.0 * P * spec.N / (enc_ms * 1e-3) / fp32_peak,
-                    "brute_force_equivalent_note": "the FP32 work a brute-force search would do in the same time; "
-                                                   "above 1 because the pruned search skips it",
-                    "hbm_gbs": (M * K * 2 + M * wpr * 4) / (enc_ms * 1e-3) / 1e9}
-    else:
-        enc_roof = brute_roof
     dec_roof = {"bound": "hbm", "achieved": dec_bytes / (dec_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": dec_bytes / (dec_ms * 1e-3) / 1e9 / hbm, "traffic": None, "kernel": "decode_tma_kernel",
                 "peak_source": f"{peak_kind} hbm_gbs", "gweights_per_s": weights / (dec_ms * 1e-3) / 1e9}
@@ -963,14 +1298,23 @@ def run_ours(args):
                "d2h_bytes_per_step": outh.numel() * 2 + pkh.numel() * 4 + 4 * M + 4 * K + 2 * K,
                "pipelining": "2 buffer slots; H2D, compute and D2H on three streams"}
 
-    # ---- oracle on the host cores (rank 0, N = 1 only)
-    cpu = None
+    # ---- the oracle on the host cores (rank 0, N = 1 only): its speed on a
+    # row sample over every core, and, in the same leg, the index parity of
+    # the whole matrix against the GPU encoding of the timed steps
+    cpu, parity = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = args.cpu_rows or auto_rows(spec)
-        times = time_oracle(W32, act, spec, C, rows, 3)
-        cpu = {"value": rows * K / statistics.median(times) / 1e9, "unit": "Gweights/s", "cores": 1,
+        pool = OraclePool()
+        try:
+            nrows, walls = time_oracle_parallel(pool, W32, act, spec, C, rows, 3)
+        finally:
+            pool.close()
+        cpu = {"value": nrows * K / statistics.median(walls) / 1e9, "unit": "Gweights/s", "cores": pool.workers,
                "kind": "oracle",
-               "sample": f"{rows} of {M} rows, calibrate + encode + decode, median of 3 (fp64 numpy, 1 thread)"}
+               "sample": f"{pool.workers} worker processes x {rows} rows of {M} per step (calibrate + encode + decode "
+                         f"of its rows, fp64 numpy, one thread each); median of 3 steps"}
+        parity = oracle_parity(W32, act, spec, C, sigma.cpu().numpy(), rnorm.cpu().numpy(), cscale.cpu().numpy(),
+                               packed.cpu().numpy().view(np.uint32))
 
     if world > 1:
         dist.barrier()
@@ -991,7 +1335,7 @@ def run_ours(args):
                    "calibrate_encode": statistics.mean(t_calenc),
                    "note": ("calibrate, encode and decode: the three separate calls (each computes s and r); "
                             "calibrate_encode: the step's fused call (s and r once)")},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 6 * args.steps, "clocks": clk,
+            "cpu_baseline": cpu, "parity": parity, "e2e": e2e, "gpu_launches": 6 * args.steps, "clocks": clk,
             "timing": ("each step replays a CUDA graph of the 6 kernels (captured once from the C-ABI calls); "
                        "'eager' is the same step launched call by call" if args.graph else
                        "each step launched call by call"),

@@ -215,6 +215,24 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
                 float *col_scale_out, int32_t *status, qamw_stream_t stream);
 
 /*
+ * qamw_encode_prepared -- qamw_encode with the channel scales and row norms
+ * given: steps (2), (3), (4) and bit packing of Methodology, reading s_j and
+ * r_i instead of computing them (steps (5) and (1)), e.g. the col_scale_out
+ * and row_norm_out of an earlier qamw_encode or qamw_calibrate_encode of the
+ * same matrix, or stored metadata. One kernel; its packed stream equals
+ * qamw_encode's bit for bit when s and r are the ones qamw_encode writes.
+ * (An interface of this library; the QAM-W page has no counterpart.)
+ *   col_scale: device float32 [K] (s_j)   row_norm: device float32 [M] (r_i; a zero
+ *              row codes x = 0, a non-finite one sets QAMW_STATUS_NONFINITE_INPUT)
+ *   other arguments as qamw_encode.
+ * Errors: QAMW_ENULL, QAMW_EINVAL (shape, code size), QAMW_EUNSUPPORTED.
+ */
+int qamw_encode_prepared(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                         const float *col_scale, const float *row_norm, int32_t block, uint64_t sign_seed,
+                         const float *sigma, const float *codebook, int32_t N, int32_t bits_per_pair,
+                         const void *search_table, uint32_t *packed_out, int32_t *status, qamw_stream_t stream);
+
+/*
  * qamw_calibrate_encode -- qamw_calibrate_sigma followed by qamw_encode on the
  * same matrix, as one call: Methodology (3) calibrates sigma over the rows of
  * W, then steps (5), (1), (2), (3), (4) code them with that sigma. The channel

@@ -219,3 +219,19 @@ def test_sharded_calibration_rejects_on_host(lib):
                                            None) == QAMW_ENULL
     assert lib.qamw_calibrate_partial_sums(FAKE, 1, 8, 256, 256, None, 0.5, 128, 1, FAKE, None, 0, None,
                                            None) == QAMW_EWORKSPACE
+
+
+def test_encode_prepared_rejects_on_host(lib):
+    def call(**kw):
+        a = dict(W=FAKE, wt=1, M=8, K=256, ldw=256, s=FAKE, r=FAKE, block=128, seed=1, sigma=FAKE, cb=FAKE,
+                 N=256, bits=8, table=None, packed=FAKE, status=None, stream=None)
+        a.update(kw)
+        return lib.qamw_encode_prepared(a["W"], a["wt"], a["M"], a["K"], a["ldw"], a["s"], a["r"], a["block"],
+                                        a["seed"], a["sigma"], a["cb"], a["N"], a["bits"], a["table"],
+                                        a["packed"], a["status"], a["stream"])
+    for kw in (dict(W=None), dict(s=None), dict(r=None), dict(sigma=None), dict(cb=None), dict(packed=None)):
+        assert call(**kw) == QAMW_ENULL
+    for kw in (dict(K=255, ldw=255), dict(block=96), dict(ldw=128), dict(bits=0), dict(N=257), dict(wt=7),
+               dict(table=ctypes.c_void_p(0x10008))):
+        assert call(**kw) == QAMW_EINVAL
+    assert call(N=16384, bits=16) == QAMW_EUNSUPPORTED

@@ -68,6 +68,13 @@ def test_fused_equals_separate_calls_bitwise(M, K, dt, block, N, bits, alpha, se
     assert sa == sb == 0
     for x, y in ((a.sigma, b.sigma), (a.row_norm, b.row_norm), (a.col_scale, b.col_scale), (a.packed, b.packed)):
         assert _same_bits(x, y)
+    # the encode kernel alone, given the scales and norms the encode wrote
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c = qamw.encode_prepared(Wd, a.col_scale, a.row_norm, block, 5, a.sigma, Cd, bits, status=st,
+                             search_table=table)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert _same_bits(a.packed, c.packed)
 
 
 def test_fused_matches_the_oracle_on_the_tiny_workload():
@@ -104,3 +111,9 @@ def test_fused_reports_bad_input_like_the_separate_calls():
     assert sa == sb and sb & qamw.STATUS_BAD_ACT_RMS and sb & qamw.STATUS_NONFINITE_NORM
     for x, y in ((a.sigma, b.sigma), (a.row_norm, b.row_norm), (a.col_scale, b.col_scale), (a.packed, b.packed)):
         assert _same_bits(x, y)
+    # the encode kernel alone reports the non-finite row norm it is given
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c = qamw.encode_prepared(Wd, a.col_scale, a.row_norm, 64, 9, a.sigma, Cd, 8, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & qamw.STATUS_NONFINITE_INPUT
+    assert _same_bits(a.packed, c.packed)

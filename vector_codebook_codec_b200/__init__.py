@@ -54,6 +54,8 @@ _SIGNATURES = {
                                    _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
     "qamw_search_cells": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p]),
+    "qamw_encode_prepared": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i32, _c_u64,
+                                            _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p]),
     "qamw_search_table_bytes": (_c_sz, [_c_i32]),
     "qamw_build_search_table": (ctypes.c_int, [_c_p, _c_i32, _c_p, _c_sz, _c_p]),
     "qamw_calibrate_sigma_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_f32,
@@ -341,6 +343,29 @@ def encode(W, act_rms, alpha: float, block: int, seed: int, sigma, codebook, bit
         _ptr(sigma), _ptr(codebook.contiguous()), N, bits, _ptr(search_table), _ptr(packed), _ptr(r), _ptr(s),
         _ptr(status), _stream_ptr(stream)))
     return Encoded(packed, r, s, sigma, M, K, block, seed, N, bits)
+
+
+def encode_prepared(W, col_scale, row_norm, block: int, seed: int, sigma, codebook, bits: int,
+                    status=None, stream=None, out=None, search_table=None) -> Encoded:
+    """Encode W given its channel scales s_j and row norms r_i (qamw_encode_prepared):
+    the encode kernel alone. ``out`` = packed words preallocated, or None."""
+    torch = _torch()
+    _need_cuda("W", W, ndim=2)
+    _need_cuda("col_scale", col_scale, torch.float32, 1)
+    _need_cuda("row_norm", row_norm, torch.float32, 1)
+    _need_cuda("sigma", sigma, torch.float32, 1)
+    _need_cuda("codebook", codebook, torch.float32, 2)
+    M, K = W.shape
+    N = codebook.shape[0]
+    wpr = words_per_row(K, bits)
+    if wpr < 0:
+        raise ValueError("invalid K / bits")
+    packed = torch.empty((M, wpr), dtype=torch.int32, device=W.device) if out is None else out
+    _check("qamw_encode_prepared", load_library().qamw_encode_prepared(
+        _ptr(W), _wdtype(W), M, K, _ld(W), _ptr(col_scale), _ptr(row_norm), block, seed & (2**64 - 1),
+        _ptr(sigma), _ptr(codebook.contiguous()), N, bits, _ptr(search_table), _ptr(packed), _ptr(status),
+        _stream_ptr(stream)))
+    return Encoded(packed, row_norm, col_scale, sigma, M, K, block, seed, N, bits)
 
 
 def calibrate_encode(W, act_rms, alpha: float, block: int, seed: int, codebook, bits: int,

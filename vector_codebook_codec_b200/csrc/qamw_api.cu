@@ -273,6 +273,36 @@ int qamw_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t
   return QAMW_OK;
 }
 
+int qamw_encode_prepared(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
+                         const float *col_scale, const float *row_norm, int32_t block, uint64_t sign_seed,
+                         const float *sigma, const float *codebook, int32_t N, int32_t bits_per_pair,
+                         const void *search_table, uint32_t *packed_out, int32_t *status, qamw_stream_t stream) {
+  static const char *fn = "qamw_encode_prepared";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  int rc;
+  if (!W || !col_scale || !row_norm || !sigma || !codebook || !packed_out)
+    return fail(QAMW_ENULL, "%s: W, col_scale, row_norm, sigma, codebook, packed_out must be non-NULL", fn);
+  if ((rc = check_dtype(w_dtype, fn))) return rc;
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if ((rc = check_code(N, bits_per_pair, fn))) return rc;
+  if (ldw < K) return fail(QAMW_EINVAL, "%s: ldw (%lld) < K (%lld)", fn, (long long)ldw, (long long)K);
+  if (search_table != nullptr && reinterpret_cast<uintptr_t>(search_table) % 16)
+    return fail(QAMW_EINVAL, "%s: search_table must be 16-byte aligned", fn);
+  EncodeArgs ea;
+  ea.rot = RotateArgs{W, w_dtype, M, K, ldw, log2i(block), sign_seed, col_scale, row_norm};
+  ea.sigma = sigma;
+  ea.codebook = codebook;
+  ea.N = N;
+  ea.bits = bits_per_pair;
+  ea.wpr = qamw_words_per_row(K, bits_per_pair);
+  ea.packed = packed_out;
+  ea.table = search_table;
+  ea.status = status;
+  cudaError_t e = launch_encode(ea, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
 int qamw_calibrate_encode(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, int64_t ldw,
                           const float *act_rms, float alpha, int32_t block, uint64_t sign_seed,
                           const float *codebook, int32_t N, int32_t bits_per_pair, const void *search_table,
