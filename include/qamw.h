@@ -325,6 +325,28 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
                 qamw_stream_t stream);
 
 /*
+ * qamw_decode_matmul -- Methodology (6) Decoding fused with the matrix
+ * multiply that consumes the weights ("Significance and Claims": the decoded
+ * weights are rounded to BF16 and fed to the matmul; the bit savings reach
+ * latency once decoding is fused into it):
+ *   Y[t][m] = sum_k X[t][k] * RN_bf16(w_hat[m][k])     (fp32 accumulation),
+ * w_hat as qamw_decode computes it. The weights are decoded tile by tile into
+ * shared memory and multiplied on the tensor cores (tcgen05, accumulators in
+ * tensor memory); they are never written to device memory.
+ *   packed, row_norm, sigma, col_scale, codebook: as qamw_decode
+ *   X : device bf16 [T][ldx] (activations, row-major; 16-byte aligned, ldx a multiple of 8)
+ *   Y : device float32 [T][ldy] (written for t < T, m < M)
+ * Limits of this build: K a multiple of 128, block <= 128, N <= 2048
+ * (QAMW_EUNSUPPORTED otherwise). Status bits as qamw_decode, plus
+ * QAMW_STATUS_TIMEOUT if a bounded wait for a copy or a tensor-core result ran out.
+ * Errors: QAMW_ENULL, QAMW_EINVAL (shape, T < 1, ldx / ldy, alignment), QAMW_EUNSUPPORTED.
+ */
+int qamw_decode_matmul(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
+                       int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
+                       int32_t bits_per_pair, const void *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
+                       int32_t *status, qamw_stream_t stream);
+
+/*
  * qamw_rotate_rows -- the rotation alone, for tests of step (2).
  * inverse == 0: Y = H_b (d * U) / sqrt(b); inverse != 0: Y = d * (H_b U) / sqrt(b),
  * per block of b columns, in fp64 (the encode path's arithmetic).

@@ -26,7 +26,7 @@ import numpy as np
 
 __all__ = [
     "MatrixSpec", "Workload", "make_matrix", "make_act_rms", "make_indices",
-    "make_row_norms", "make_sigma", "to_bf16", "tiny", "llama7b_attn", "mlp_runs",
+    "make_row_norms", "make_sigma", "make_activations", "to_bf16", "tiny", "llama7b_attn", "mlp_runs",
     "stack_1p1b", "decode_sweep_13b", "rate_variant", "gaussian_points", "WORKLOADS",
 ]
 
@@ -99,6 +99,12 @@ def make_indices(M: int, P: int, N: int, seed: int) -> np.ndarray:
 def make_row_norms(M: int, seed: int) -> np.ndarray:
     """Positive float32 row norms ~ 0.02*sqrt(K)-sized, for decode-only inputs."""
     return (np.exp(_rng(seed + 1).standard_normal(M) * 0.25) * 1.0).astype(np.float32)
+
+
+def make_activations(T: int, K: int, seed: int) -> np.ndarray:
+    """Activations for the fused decode + matmul, N(0, 1) float32 [T, K] (rounded
+    to bf16 by the caller where the kernel reads bf16)."""
+    return _rng(seed + 11).standard_normal((T, K), dtype=np.float32)
 
 
 def gaussian_points(T: int, seed: int) -> np.ndarray:

@@ -54,6 +54,8 @@ _SIGNATURES = {
                                    _c_i32, _c_p, ctypes.c_int, _c_i64, _c_p, _c_p]),
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
     "qamw_search_cells": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p]),
+    "qamw_decode_matmul": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
+                                          _c_i32, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p]),
     "qamw_encode_prepared": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i32, _c_u64,
                                             _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p]),
     "qamw_search_table_bytes": (_c_sz, [_c_i32]),
@@ -439,6 +441,23 @@ def decode(enc: Encoded, codebook, out_dtype=None, status=None, stream=None, out
         enc.block, enc.seed & (2**64 - 1), _ptr(codebook.contiguous()), codebook.shape[0], enc.bits,
         _ptr(out), ot, _ld(out), _ptr(status), _stream_ptr(stream)))
     return out
+
+
+def decode_matmul(enc: Encoded, codebook, X, status=None, stream=None, out=None):
+    """Y = X @ RN_bf16(decode(enc))^T with the decode fused into the tensor-core
+    matmul (qamw_decode_matmul); X is a bf16 CUDA tensor [T, K], Y float32 [T, M]."""
+    torch = _torch()
+    _need_cuda("codebook", codebook, torch.float32, 2)
+    _need_cuda("X", X, torch.bfloat16, 2)
+    if X.shape[1] != enc.K:
+        raise ValueError("X must have K columns")
+    T = X.shape[0]
+    Y = torch.empty((T, enc.M), dtype=torch.float32, device=X.device) if out is None else out
+    _check("qamw_decode_matmul", load_library().qamw_decode_matmul(
+        _ptr(enc.packed), _ptr(enc.row_norm), _ptr(enc.sigma), _ptr(enc.col_scale), enc.M, enc.K, enc.block,
+        enc.seed & (2**64 - 1), _ptr(codebook.contiguous()), codebook.shape[0], enc.bits, _ptr(X), T, _ld(X),
+        _ptr(Y), _ld(Y), _ptr(status), _stream_ptr(stream)))
+    return Y
 
 
 def rotate_rows(U, block: int, seed: int, inverse: bool = False, stream=None):

@@ -403,6 +403,46 @@ int qamw_encode_polar(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, i
   return QAMW_OK;
 }
 
+int qamw_decode_matmul(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
+                       int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
+                       int32_t bits_per_pair, const void *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
+                       int32_t *status, qamw_stream_t stream) {
+  static const char *fn = "qamw_decode_matmul";
+  CallRange nvtx_range(fn);
+  g_last_error[0] = 0;
+  int rc;
+  if (!packed || !row_norm || !sigma || !codebook || !X || !Y)
+    return fail(QAMW_ENULL, "%s: packed, row_norm, sigma, codebook, X and Y must be non-NULL", fn);
+  if ((rc = check_shape(M, K, block, fn))) return rc;
+  if ((rc = check_code(N, bits_per_pair, fn))) return rc;
+  if (T < 1) return fail(QAMW_EINVAL, "%s: T (%lld) must be >= 1", fn, (long long)T);
+  if (ldx < K || ldy < M)
+    return fail(QAMW_EINVAL, "%s: ldx (%lld) must be >= K and ldy (%lld) >= M", fn, (long long)ldx, (long long)ldy);
+  if (K % 128 != 0 || block > 128 || N > 2048 || T > (int64_t)1 << 30)
+    return fail(QAMW_EUNSUPPORTED, "%s: needs K a multiple of 128, block <= 128, N <= 2048, T <= 2^30", fn);
+  if (reinterpret_cast<uintptr_t>(X) % 16 != 0 || ldx % 8 != 0)
+    return fail(QAMW_EINVAL, "%s: X must be 16-byte aligned with ldx a multiple of 8", fn);
+  DecodeArgs a;
+  a.packed = packed;
+  a.row_norm = row_norm;
+  a.sigma = sigma;
+  a.col_scale = col_scale;
+  a.M = M;
+  a.K = K;
+  a.log2b = log2i(block);
+  a.seed = sign_seed;
+  a.codebook = codebook;
+  a.N = N;
+  a.bits = bits_per_pair;
+  a.wpr = qamw_words_per_row(K, bits_per_pair);
+  a.out = nullptr;
+  a.out_t = QAMW_BF16;
+  a.ldo = 0;
+  a.status = status;
+  cudaError_t e = launch_decode_gemm(a, static_cast<const uint16_t *>(X), T, ldx, Y, ldy, (cudaStream_t)stream);
+  return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
 int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
                 int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
                 int32_t bits_per_pair, void *W_out, qamw_dtype out_dtype, int64_t ldo, int32_t *status,

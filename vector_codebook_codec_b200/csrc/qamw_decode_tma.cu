@@ -35,6 +35,7 @@
 #include "qamw_device.cuh"
 #include "qamw_internal.h"
 #include "qamw_mbarrier.cuh"
+#include "qamw_tensor_map.h"
 
 namespace qamw {
 namespace {
@@ -355,6 +356,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 // --------------------------------------------------------------------------
 // host side
 // --------------------------------------------------------------------------
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -367,6 +370,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   });
   return fn;
 }
+
+namespace {
 
 template <int BITS, int LB>
 cudaError_t launch_tma_t(const DecodeArgs &a, cudaStream_t s) {
