@@ -57,14 +57,15 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="llama7b_attn",
                    choices=("llama7b_attn", "tiny", "decode_13b", "rate35", "rate4", "lloyd", "polar", "mlp",
-                            "stack_1p1b"),
+                            "stack_1p1b", "decode_gemm"),
                    help="llama7b_attn: 4096x4096 bf16 at 2048 centroids (5.5 bits/weight; the default); "
                         "rate35 / rate4: the same matrix at 128 / 256 centroids (3.5 / 4 bits/weight); "
                         "decode_13b: decode-only sweep over the 13B shapes; tiny: 256x512 fp32; "
                         "lloyd: codebook training, one Lloyd iteration of 2048 centroids on 2^21 samples per step; "
                         "polar: the polar baseline codec on the 4096x4096 projection at 2048 points; "
                         "mlp: the 24 MLP runs (11008x4096 and 4096x11008, alpha x block x codebook); "
-                        "stack_1p1b: the 154 matrices of the 22-layer 1.1B-shaped stack")
+                        "stack_1p1b: the 154 matrices of the 22-layer 1.1B-shaped stack; "
+                        "decode_gemm: the fused decode + matmul on the 13824x5120 matrix at 1..4096 tokens")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="rows per oracle sample (0 = auto)")
@@ -306,6 +307,27 @@ def run_reference_special(args):
         return _reference_line(args, "QAM-W codebook training: Lloyd iterations per second", value, "iterations/s",
                                {"workload": "lloyd_N2048_T2097152", "N": LLOYD_N, "T": LLOYD_T},
                                f"{Ts} of {LLOYD_T} samples per iteration, scaled", 1e3 / value, os.cpu_count())
+    if args.workload == "decode_gemm":
+        spec = synth.decode_sweep_13b().specs[1]
+        rows = args.cpu_rows or 8
+        C = q.load_codebook(spec.N)
+        idx = synth.make_indices(rows, spec.K // 2, spec.N, spec.seed)
+        r = synth.make_row_norms(rows, spec.seed)
+        sig = synth.make_sigma(spec.K // 2, spec.seed)
+        s_ = synth.make_act_rms(spec.K, 0.5, spec.seed)
+        X = synth.make_activations(1, spec.K, 901).astype(np.float64)
+        ts = []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            Wh = codec.decode_with_scale(idx, r, sig, s_, spec.K, spec.block, spec.seed, C)
+            X @ Wh.T
+            if i >= args.warmup:
+                ts.append(time.perf_counter() - t0)
+        value = rows * spec.K * len(ts) / sum(ts) / 1e9
+        return _reference_line(args, METRIC, value, "Gweights/s",
+                               {"workload": "decode_gemm_13824x5120_bf16_b128_N2048", "op": "decode then X W^T"},
+                               f"{rows} of {spec.M} rows per step, decoded and multiplied with one token",
+                               1e3 * sum(ts) / len(ts))
     if args.workload == "polar":
         spec = synth.llama7b_attn().specs[0]
         _, W32 = synth.to_bf16(synth.make_matrix(spec))
@@ -354,7 +376,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    if args.workload in ("lloyd", "polar", "decode_13b"):
+    if args.workload in ("lloyd", "polar", "decode_13b", "decode_gemm"):
         print(json.dumps(run_reference_special(args)), flush=True)
         return 0
     import synth
@@ -998,7 +1020,132 @@ def run_multi(args):
     return 0
 
 
+DG_TOKENS = (1, 16, 128, 4096)
+
+
+def run_decode_gemm(args):
+    """The fused decode + matmul (qamw_decode_matmul) on the 13B up projection
+    (13824 x 5120, 2048 centroids, block 128), pre-encoded: Y = X W^T for T in
+    {1, 16, 128, 4096} tokens, against the unfused path (qamw_decode to bf16,
+    then torch's bf16 matmul, i.e. cuBLAS) and against cuBLAS alone on the
+    already-decoded bf16 weights. A step runs every T once; the headline is
+    the fused call's weight throughput at T = 1 (memory-bound: 0.69 bytes per
+    weight read instead of 2)."""
+    import torch
+    import synth
+    import vector_codebook_codec_b200 as q
+    from vector_codebook_codec_b200 import build as qbuild
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qbuild.build()
+    spec = synth.decode_sweep_13b().specs[1]
+    M, K = spec.M, spec.K
+    # pre-encode the matrix with the GPU encode (as the decode-only workload does)
+    Wt, _ = synth.to_bf16(synth.make_matrix(spec))
+    Wd = Wt.to(dev)
+    act = torch.from_numpy(synth.act_for(spec)).to(dev)
+    Cd = torch.from_numpy(q.load_codebook(spec.N)).to(dev)
+    sig = q.calibrate_sigma(Wd, act, spec.alpha, spec.block, spec.seed)
+    enc = q.encode(Wd, act, spec.alpha, spec.block, spec.seed, sig, Cd, spec.bits,
+                   search_table=q.build_search_table(Cd))
+    del Wd
+    Wb = q.decode(enc, Cd, out_dtype=torch.bfloat16)          # for the cuBLAS-only reference
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    Xs = {T: torch.from_numpy(synth.make_activations(T, K, 900 + T)).to(torch.bfloat16).to(dev) for T in DG_TOKENS}
+    Ys = {T: torch.empty((T, M), dtype=torch.float32, device=dev) for T in DG_TOKENS}
+    Wtmp = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+
+    def fused(T):
+        q.decode_matmul(enc, Cd, Xs[T], status=status, out=Ys[T])
+
+    def unfused(T):
+        q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=Wtmp)
+        torch.matmul(Xs[T], Wtmp.T)
+
+    def cublas(T):
+        torch.matmul(Xs[T], Wb.T)
+
+    def timed(fn, T, reps):
+        ts = []
+        for i in range(reps):
+            flush.fill_(float(i))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(T)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    for T in DG_TOKENS:
+        for fn in (fused, unfused, cublas):
+            for _ in range(args.warmup):
+                fn(T)
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()} after warm-up")
+    # correctness at the smallest and largest T: fused vs unfused (same bf16 weights, fp32 accumulation)
+    for T in (DG_TOKENS[0], DG_TOKENS[-1]):
+        fused(T)
+        ref = torch.matmul(Xs[T].float(), Wb.float().T)
+        scale = torch.matmul(Xs[T].float().abs(), Wb.float().abs().T)
+        if not bool(((Ys[T] - ref).abs() <= 2.0 ** -7 * scale + 1e-6).all()):
+            raise SystemExit(f"fused decode + matmul differs from decode + matmul at T={T}")
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    rows = []
+    total_ms = 0.0
+    for T in DG_TOKENS:
+        reps = max(args.steps, 3)
+        tf, tu, tc = timed(fused, T, reps), timed(unfused, T, reps), timed(cublas, T, reps)
+        total_ms += tf
+        rows.append({"tokens": T, "fused_us": 1e3 * tf, "decode_then_cublas_us": 1e3 * tu,
+                     "cublas_on_decoded_bf16_us": 1e3 * tc, "fused_speedup_vs_unfused": tu / tf,
+                     "fused_tflops": 2.0 * M * K * T / (tf * 1e-3) / 1e12})
+    time.sleep(0.2)
+    clk = clocks.stop()
+    if status.item() != 0:
+        raise SystemExit(f"device status {status.item()} in the timed calls")
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    tc_peak = float(peaks.get("bf16_tflops", 1590.0))
+    wpr = q.words_per_row(K, spec.bits)
+    t1 = rows[0]["fused_us"] * 1e-6
+    bytes1 = M * wpr * 4 + 4 * M + 4 * K + 2 * K + 8 * spec.N + 2 * K + 4 * M
+    t4 = rows[-1]["fused_us"] * 1e-6
+    flops4 = 2.0 * M * K * DG_TOKENS[-1]
+    value = M * K / t1 / 1e9
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; no checkpoint)",
+                "config": {"workload": "decode_gemm_13824x5120_bf16_b128_N2048", "M": M, "K": K, "N": spec.N,
+                           "bits": spec.bits, "tokens": list(DG_TOKENS),
+                           "op": "Y[T x M] = X[T x K] decode(W)^T, fp32 accumulation",
+                           "l2": "flushed by a 256 MiB write before every timed call",
+                           "value_note": "weights per second of the fused call at T = 1"},
+                "roofline": {"bound": "hbm", "achieved": bytes1 / t1 / 1e9, "peak": hbm, "unit": "GB/s",
+                             "frac": bytes1 / t1 / 1e9 / hbm, "traffic": None,
+                             "kernel": "decode_gemm_kernel at T = 1 (packed words, r, sigma, s, codebook, x, y)",
+                             "peak_source": f"{peak_kind} hbm_gbs"},
+                "rooflines": {"tensor_at_4096_tokens": {
+                    "bound": "tensor", "achieved": flops4 / t4 / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": flops4 / t4 / 1e12 / tc_peak, "traffic": None,
+                    "kernel": "decode_gemm_kernel at T = 4096", "peak_source": f"{peak_kind} bf16_tflops (burst)"}},
+                "per_tokens": rows, "gpu_launches": len(DG_TOKENS) * 2 * max(args.steps, 3) + len(DG_TOKENS) * max(args.steps, 3),
+                "clocks": clk, "cpu_baseline": None, "e2e": None,
+                "timing": "each call timed alone with events after an L2 flush; median of the repetitions"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args):
+    if args.workload == "decode_gemm":
+        return run_decode_gemm(args)
     if args.workload in ("mlp", "stack_1p1b"):
         return run_multi(args)
     if args.workload == "polar":

@@ -335,6 +335,7 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
  * tensor memory); they are never written to device memory.
  *   packed, row_norm, sigma, col_scale, codebook: as qamw_decode
  *   X : device bf16 [T][ldx] (activations, row-major; 16-byte aligned, ldx a multiple of 8)
+ *   (packed must be 8-byte and sigma 16-byte aligned)
  *   Y : device float32 [T][ldy] (written for t < T, m < M)
  * Limits of this build: K a multiple of 128, block <= 128, N <= 2048
  * (QAMW_EUNSUPPORTED otherwise). Status bits as qamw_decode, plus

@@ -20,7 +20,7 @@ def _run(argv):
     return rc, [ln for ln in out.getvalue().splitlines() if ln.strip()]
 
 
-@pytest.mark.parametrize("workload,rows", [("tiny", 4), ("polar", 2), ("decode_13b", 1), ("stack_1p1b", 1)])
+@pytest.mark.parametrize("workload,rows", [("tiny", 4), ("polar", 2), ("decode_13b", 1), ("stack_1p1b", 1), ("decode_gemm", 1)])
 def test_reference_arm_prints_one_contract_line(monkeypatch, workload, rows):
     monkeypatch.delenv("RANK", raising=False)
     monkeypatch.delenv("WORLD_SIZE", raising=False)

@@ -422,6 +422,8 @@ int qamw_decode_matmul(const uint32_t *packed, const float *row_norm, const floa
     return fail(QAMW_EUNSUPPORTED, "%s: needs K a multiple of 128, block <= 128, N <= 2048, T <= 2^30", fn);
   if (reinterpret_cast<uintptr_t>(X) % 16 != 0 || ldx % 8 != 0)
     return fail(QAMW_EINVAL, "%s: X must be 16-byte aligned with ldx a multiple of 8", fn);
+  if (reinterpret_cast<uintptr_t>(packed) % 8 != 0 || reinterpret_cast<uintptr_t>(sigma) % 16 != 0)
+    return fail(QAMW_EINVAL, "%s: packed must be 8-byte and sigma 16-byte aligned", fn);
   DecodeArgs a;
   a.packed = packed;
   a.row_norm = row_norm;

@@ -36,7 +36,7 @@ namespace {
 
 constexpr int kBM = 128;              // output rows per CTA (tensor-memory lanes)
 constexpr int kBK = 128;              // columns per chunk (whole Hadamard blocks, b <= 128)
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;            // one (row, 32-column quarter) of the chunk per thread
 constexpr int kThreads = kWarps * 32;
 constexpr int kAtomBytesA = kBM * 128;                // one 64-column swizzle atom of the weight tile
 constexpr int kStageBytesA = 2 * kAtomBytesA;         // 128 columns = 2 atoms
@@ -49,6 +49,26 @@ struct GemmArgs {
   float *Y;              // [T][ldy] fp32
   int64_t ldy;
 };
+
+// shared-memory layout after the 1024-aligned operand stages
+struct GemmSmem {
+  int stage_b, words_row, words_stage;
+  size_t off_b, off_words, off_cb, off_fac, off_sig, total;
+};
+constexpr int kWordStages = 3;   // packed words of a chunk are fetched two chunks ahead
+__host__ __device__ __forceinline__ GemmSmem gemm_smem(int NT, int N, int B, int64_t K) {
+  GemmSmem g;
+  g.stage_b = NT * 256;                          // 2 atoms of NT rows x 128 B
+  g.words_row = 2 * B;                           // a row's packed words of one chunk (64 pairs)
+  g.words_stage = kBM * g.words_row + 4;         // + 4: the unpacking reads one word past a row
+  g.off_b = 2 * (size_t)kStageBytesA;
+  g.off_words = g.off_b + 2 * (size_t)g.stage_b;
+  g.off_cb = g.off_words + kWordStages * (size_t)g.words_stage * 4;
+  g.off_fac = (g.off_cb + (size_t)N * 8 + 15) & ~(size_t)15;   // 16-byte loads of the factors
+  g.off_sig = g.off_fac + (size_t)K * 4;                        // every column's factor, computed once
+  g.total = g.off_sig + kWordStages * (kBK / 2) * 4;
+  return g;
+}
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   // start address >> 4 | leading offset 16 B (ignored for swizzled K-major) |
@@ -97,27 +117,59 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Index of pair kk of a row (LSB-first stream of B-bit fields).
-__device__ __forceinline__ uint32_t unpack_index(const uint32_t *row, int64_t kk, int B) {
-  const int64_t bit = kk * B;
-  const int64_t w = bit >> 5;
-  const int off = (int)(bit & 31);
-  uint64_t v = row[w];
-  if (off + B > 32) v |= (uint64_t)row[w + 1] << 32;
-  return (uint32_t)(v >> off) & ((1u << B) - 1u);
+// The 16 indices of pairs 16 q .. 16 q + 15 of a row's chunk, from its 2B
+// staged words (LSB-first B-bit fields). BB > 0: B fixed at compile time (the
+// quarter's first field starts at bit 0 or 16 of a word; a 16-bit funnel
+// shift aligns it, and every later position is a constant).
+template <int BB>
+__device__ __forceinline__ void unpack16(const uint32_t *rw, int q, int B, uint32_t (&idx)[16]) {
+  if (BB > 0) {
+    constexpr int kNW = (16 * BB + 31) / 32 + 1;
+    const int bit0 = 16 * q * BB;
+    const uint32_t *p = rw + (bit0 >> 5);
+    uint32_t w[kNW + 1];
+#pragma unroll
+    for (int i = 0; i <= kNW; ++i) w[i] = p[i];
+    if (bit0 & 31) {
+#pragma unroll
+      for (int i = 0; i < kNW; ++i) w[i] = __funnelshift_r(w[i], w[i + 1], 16);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int b = k * BB, wi = b >> 5, sh = b & 31;
+      uint32_t v = w[wi] >> sh;
+      if (sh + BB > 32) v |= w[wi + 1] << (32 - sh);
+      idx[k] = v & ((1u << BB) - 1u);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int b = (16 * q + k) * B, wi = b >> 5, sh = b & 31;
+      uint64_t v = rw[wi];
+      if (sh + B > 32) v |= (uint64_t)rw[wi + 1] << 32;
+      idx[k] = (uint32_t)(v >> sh) & ((1u << B) - 1u);
+    }
+  }
 }
 
+// BB > 0 fixes the code size, LB > 0 log2 b, at compile time (a butterfly
+// stage guarded by a run-time block size costs register copies where the two
+// paths join); 0 reads them at run time.
+template <int BB, int LB>
 __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs g) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   // 1024-byte alignment for the swizzled operand tiles
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const DecodeArgs &a = g.d;
   const int NT = g.NT;
-  const int stage_b = NT * 256;                 // 2 atoms of NT rows x 128 B
-  unsigned char *A0 = smem;                     // [2][kStageBytesA]
-  unsigned char *B0 = smem + 2 * kStageBytesA;  // [2][stage_b]
-  float2 *cb = reinterpret_cast<float2 *>(B0 + 2 * stage_b);
-  float *fac = reinterpret_cast<float *>(cb + a.N);   // [kBK] d_j / (sqrt(b) s_j) of the chunk
+  const int B = BB > 0 ? BB : a.bits;
+  const GemmSmem L = gemm_smem(NT, a.N, B, a.K);
+  unsigned char *A0 = smem;                                          // [2][kStageBytesA]
+  unsigned char *B0 = smem + L.off_b;                                // [2][stage_b]
+  uint32_t *W0 = reinterpret_cast<uint32_t *>(smem + L.off_words);   // [2][words_stage] packed words of a chunk
+  float2 *cbf = reinterpret_cast<float2 *>(smem + L.off_cb);         // (c0 + c1, c0 - c1): the first butterfly folded in
+  float *fac = reinterpret_cast<float *>(smem + L.off_fac);          // [K] d_j / (sqrt(b) s_j)
+  float *S0 = reinterpret_cast<float *>(smem + L.off_sig);           // [kWordStages][64] sigma of a chunk
 
   __shared__ __align__(8) uint64_t bar_x[2], bar_mma[2];
   __shared__ uint32_t s_tmem;
@@ -127,12 +179,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
   const int64_t m0 = (int64_t)blockIdx.x * kBM;
   const int64_t t0 = (int64_t)blockIdx.y * NT;
   const int64_t n_chunks = a.K / kBK;
-  const int B = a.bits;
-  const int log2b = a.log2b;
-  const double inv_sqrt_b = 1.0 / sqrt((double)(1 << log2b));
+  const int log2b = LB > 0 ? LB : a.log2b;
+  const float inv_sqrt_b = (float)(1.0 / sqrt((double)(1 << log2b)));
   const uint32_t tmem_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
 
-  for (int i = threadIdx.x; i < a.N; i += kThreads) cb[i] = make_float2(a.codebook[2 * i], a.codebook[2 * i + 1]);
+  // packed words and sigma of chunk c into staging buffer c % 3 (cp.async, 8 bytes
+  // at a time: a row's 2B words of a chunk start 8B-byte aligned; four threads
+  // per row; rows past M read as 0)
+  auto stage_chunk = [&](int64_t c) {
+    const int ws = (int)(c % kWordStages);
+    uint32_t *dw = W0 + ws * L.words_stage;
+    const int row = threadIdx.x >> 2, part = threadIdx.x & 3;
+    const int64_t m = m0 + row;
+    uint32_t *drow = dw + row * L.words_row;
+    if (m < a.M) {
+      const uint32_t *src = a.packed + m * a.wpr + c * L.words_row;
+      for (int k = part; k < B; k += 4) cp_async8(drow + 2 * k, src + 2 * k);
+    } else {
+      for (int k = part; k < B; k += 4) *reinterpret_cast<uint2 *>(drow + 2 * k) = make_uint2(0u, 0u);
+    }
+    if (threadIdx.x < kBK / 8)
+      cp_async16(S0 + ws * (kBK / 2) + 4 * threadIdx.x, a.sigma + c * (kBK / 2) + 4 * threadIdx.x);
+    cp_async_commit();
+  };
+
+  for (int i = threadIdx.x; i < a.N; i += kThreads) {
+    const float c0 = a.codebook[2 * i], c1 = a.codebook[2 * i + 1];
+    cbf[i] = make_float2(c0 + c1, c0 - c1);
+  }
+  if (threadIdx.x < 4 * kWordStages) {   // the padding words past the last row of each staging buffer
+    W0[(threadIdx.x >> 2) * L.words_stage + kBM * L.words_row + (threadIdx.x & 3)] = 0u;
+  }
+  // every column's factor d_j / (sqrt(b) s_j), once
+  for (int64_t j = threadIdx.x; j < a.K; j += kThreads) {
+    float f = __fdiv_rn(inv_sqrt_b, a.col_scale != nullptr ? a.col_scale[j] : 1.0f);
+    if (mask_is_negative(a.seed, j)) f = -f;
+    fac[j] = f;
+  }
   if (threadIdx.x == 0) {
     mbar_init(&bar_x[0], 1);
     mbar_init(&bar_x[1], 1);
@@ -147,6 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  if (n_chunks > 0) stage_chunk(0);
+  if (n_chunks > 1) stage_chunk(1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -154,115 +239,116 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
   // instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N = NT, M = 128
   const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 
-  // the two rows a thread decodes per chunk: rows 16 w + 8 i + (lane / 4), quarter q = lane % 4
+  // this thread's item of every chunk: row rl = 8 w + lane / 4, columns 32 q .. 32 q + 31
   const int q = lane & 3;
-  uint32_t bad = 0;
-  float rn[2];
-  bool rin[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int64_t m = m0 + 16 * warp + 8 * i + (lane >> 2);
-    rin[i] = m < a.M;
-    rn[i] = rin[i] ? a.row_norm[m] : 0.0f;
-    if (rin[i] && !isfinite(rn[i])) bad |= QAMW_STATUS_NONFINITE_NORM;
-  }
+  const int rl = 8 * warp + (lane >> 2);
+  const int64_t mrow = m0 + rl;
+  const bool rin = mrow < a.M;
+  const float rn = rin ? a.row_norm[mrow] : 0.0f;
+  uint32_t bad = (rin && !isfinite(rn)) ? QAMW_STATUS_NONFINITE_NORM : 0u;
+  const bool check_idx = a.N < (1 << B);
+  unsigned char *arow0 = A0 + (q >> 1) * kAtomBytesA + rl * 128;
 
   bool failed = false;
   for (int64_t c = 0; c < n_chunks && !failed; ++c) {
     const int s = (int)(c & 1);
-    unsigned char *As = A0 + s * kStageBytesA;
-    unsigned char *Bs = B0 + s * stage_b;
-    if (c >= 2) {   // stage s was read by the MMAs of chunk c - 2
+    unsigned char *Bs = B0 + s * L.stage_b;
+    if (c >= 2) {   // stage s was read by the MMAs of chunk c - 2 (every thread waits before overwriting it)
       if (!mbar_wait(&bar_mma[s], (uint32_t)(((c - 2) >> 1) & 1), kWaitLimit)) bad |= QAMW_STATUS_TIMEOUT;
     }
-    if (__syncthreads_or(bad & QAMW_STATUS_TIMEOUT)) { failed = true; break; }
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(&bar_x[s], (uint32_t)stage_b);
+    if (threadIdx.x == 0 && !(bad & QAMW_STATUS_TIMEOUT)) {
+      mbar_arrive_expect_tx(&bar_x[s], (uint32_t)L.stage_b);
       tma_load_2d(Bs, &xmap, (int)(c * kBK), (int)t0, &bar_x[s]);
       tma_load_2d(Bs + NT * 128, &xmap, (int)(c * kBK + 64), (int)t0, &bar_x[s]);
     }
-    // the chunk's column factors d_j / (sqrt(b) s_j)
-    if (threadIdx.x < kBK) {
-      const int64_t j = c * kBK + threadIdx.x;
-      double f = inv_sqrt_b / (a.col_scale != nullptr ? (double)a.col_scale[j] : 1.0);
-      if (mask_is_negative(a.seed, j)) f = -f;
-      fac[threadIdx.x] = (float)f;
-    }
+    // the words of chunk c + 2 in flight while this one is decoded (its
+    // buffer held chunk c - 1, decoded before the previous barrier)
+    if (c + 2 < n_chunks) stage_chunk(c + 2);
+    if (c + 2 < n_chunks) cp_async_wait<2>();   // chunk c's words and sigma have landed
+    else if (c + 1 < n_chunks) cp_async_wait<1>();
+    else cp_async_wait<0>();
     __syncthreads();
-#pragma unroll 1
-    for (int i = 0; i < 2; ++i) {
-      const int rl = 16 * warp + 8 * i + (lane >> 2);
-      const int64_t m = m0 + rl;
-      float v[32];
-      if (rin[i]) {
-        const uint32_t *prow = a.packed + m * a.wpr;
+
+    const int ws = (int)(c % kWordStages);
+    const uint32_t *rw = W0 + ws * L.words_stage + rl * L.words_row;
+    const float4 *sg4 = reinterpret_cast<const float4 *>(S0 + ws * (kBK / 2) + 16 * q);
+    uint32_t idx[16];
+    unpack16<BB>(rw, q, B, idx);
+    if (check_idx) {   // a codebook smaller than 2^B: out-of-range indices decode as centroid 0
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        if (idx[p] >= (uint32_t)a.N) { bad |= QAMW_STATUS_BAD_INDEX; idx[p] = 0; }
+      }
+    }
+    float2 v[16];   // v[p] = r sigma_k (c0 + c1, c0 - c1): block bit 0 done, the row norm applied
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 sk = sg4[h];
+      const float sr[4] = {sk.x * rn, sk.y * rn, sk.z * rn, sk.w * rn};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[4 * h + u] = mul2(cbf[idx[4 * h + u]], make_float2(sr[u], sr[u]));
+    }
+    // block bits 1..4 in registers (pairs p and p | h/2), 5..6 across the 4 lanes of the row
+#pragma unroll
+    for (int t = 1; t < 5; ++t) {
+      if (t < log2b) {
+        const int h = 1 << (t - 1);
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
-          const int64_t kk = c * (kBK / 2) + 16 * q + p;
-          uint32_t idx = unpack_index(prow, kk, B);
-          if (idx >= (uint32_t)a.N) { bad |= QAMW_STATUS_BAD_INDEX; idx = 0; }
-          const float2 cc = cb[idx];
-          const float sg = a.sigma[kk];
-          v[2 * p] = cc.x * sg;
-          v[2 * p + 1] = cc.y * sg;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
-      }
-      // inverse Hadamard butterflies: block bits 0..4 in registers, 5..6 across lanes
-#pragma unroll
-      for (int t = 0; t < 5; ++t) {
-        if (t < log2b) {
-          const int h = 1 << t;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if ((e & h) == 0) {
-              const float x0 = v[e], x1 = v[e | h];
-              v[e] = x0 + x1;
-              v[e | h] = x0 - x1;
-            }
+          if ((p & h) == 0) {
+            const float2 x0 = v[p], x1 = v[p | h];
+            v[p] = add2(x0, x1);
+            v[p | h] = sub2(x0, x1);
           }
         }
       }
+    }
 #pragma unroll
-      for (int t = 5; t < 7; ++t) {
-        if (t < log2b) {
-          const int hb = 1 << (t - 5);
-          const float sgn = (lane & hb) ? -1.0f : 1.0f;
+    for (int t = 5; t < 7; ++t) {
+      if (t < log2b) {
+        const int hb = 1 << (t - 5);
+        const float sgn = (lane & hb) ? -1.0f : 1.0f;
+        const float2 sg2 = make_float2(sgn, sgn);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __fmaf_rn(sgn, v[e], __shfl_xor_sync(0xffffffffu, v[e], hb));
+        for (int p = 0; p < 16; ++p) {
+          const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[p].x, hb), __shfl_xor_sync(0xffffffffu, v[p].y, hb));
+          v[p] = fma2(sg2, v[p], o);
         }
       }
-      // scale, round to bf16 and store into the swizzled K-major tile:
-      // row rl, columns 32 q .. 32 q + 31 = atom q / 2, 16-byte chunks 4 (q % 2) .. + 3
-      const float r = rn[i];
-      unsigned char *arow = As + (q >> 1) * kAtomBytesA + rl * 128;
+    }
+    if (!rin) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t pk[4];
+      for (int p = 0; p < 16; ++p) v[p] = make_float2(0.0f, 0.0f);
+    }
+    // scale by r d_j / (sqrt(b) s_j), round to bf16, store into the swizzled K-major tile:
+    // row rl, columns 32 q .. 32 q + 31 = atom q / 2, 16-byte chunks 4 (q % 2) .. + 3
+    unsigned char *arow = arow0 + s * kStageBytesA;
+    const float4 *f4 = reinterpret_cast<const float4 *>(fac + c * kBK + 32 * q);
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int e = 8 * ch + 2 * h;
-          const float w0 = (v[e] * r) * fac[32 * q + e];
-          const float w1 = (v[e + 1] * r) * fac[32 * q + e + 1];
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(w0, w1);
-          pk[h] = *reinterpret_cast<const uint32_t *>(&b2);
-        }
-        const int chunk16 = 4 * (q & 1) + ch;
-        *reinterpret_cast<uint4 *>(arow + ((chunk16 ^ (rl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float4 f = f4[2 * ch + h];
+        const float2 w0 = mul2(v[4 * ch + 2 * h], make_float2(f.x, f.y));
+        const float2 w1 = mul2(v[4 * ch + 2 * h + 1], make_float2(f.z, f.w));
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(w0.x, w0.y), b1 = __floats2bfloat162_rn(w1.x, w1.y);
+        pk[2 * h] = *reinterpret_cast<const uint32_t *>(&b0);
+        pk[2 * h + 1] = *reinterpret_cast<const uint32_t *>(&b1);
       }
+      const int chunk16 = 4 * (q & 1) + ch;
+      *reinterpret_cast<uint4 *>(arow + ((chunk16 ^ (rl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
     fence_proxy_async_smem();   // the tile's generic stores become visible to the tensor cores
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(bad & QAMW_STATUS_TIMEOUT)) { failed = true; break; }
     if (threadIdx.x == 0) {
       if (!mbar_wait(&bar_x[s], (uint32_t)((c >> 1) & 1), kWaitLimit)) {
         bad |= QAMW_STATUS_TIMEOUT;
         s_fail = 1;
       } else {
         tc_fence_after();
-        const uint32_t a_base = smem_u32(As), b_base = smem_u32(Bs);
+        const uint32_t a_base = smem_u32(A0 + s * kStageBytesA), b_base = smem_u32(Bs);
 #pragma unroll
         for (int k16 = 0; k16 < kBK / 16; ++k16) {
           const uint32_t atom = k16 >> 2, koff = (k16 & 3) * 32;
@@ -274,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
       }
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
   if (s_fail) failed = true;
   // the last chunk's commit covers every MMA before it
@@ -287,15 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
   failed = __syncthreads_or(failed ? 1 : 0) != 0;
   if (!failed) {
     tc_fence_after();
-    // warps w and w + 4 read tensor-memory lanes 32 (w % 4) .. + 31 (rows), each half of the columns
-    const int wq = warp & 3;
+    // warps w, w + 4, w + 8, w + 12 read tensor-memory lanes 32 (w % 4) .. + 31 (rows), a quarter of the columns each
+    const int wq = warp & 3, grp = warp >> 2;
     const int64_t m = m0 + 32 * wq + lane;
-    const int half = warp >> 2;
-    const int ncol = NT / 2;   // a multiple of 8
-    const int cend = (half + 1) * ncol;
-    // 16 columns per load; a load may reach 8 columns past the half (never
-    // past the allocated columns: NT + 8 <= the allocation for NT = 16 * odd)
-    for (int c0 = half * ncol; c0 < cend; c0 += 16) {
+    const int ncol = NT / 4;   // a multiple of 4
+    const int cbeg = grp * ncol, cend = cbeg + ncol;
+    // 16 columns per load; a load may reach 12 columns past the quarter (never
+    // past the allocated columns, which exceed NT by at least 16 unless the quarters are multiples of 16)
+    for (int c0 = cbeg; c0 < cend; c0 += 16) {
       float v[16];
       tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)c0, v);
 #pragma unroll
@@ -321,15 +407,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
 
 }  // namespace
 
-size_t decode_gemm_smem_bytes(int NT, int N) {
-  return 1024 + 2 * (size_t)kStageBytesA + 2 * (size_t)NT * 256 + (size_t)N * 8 + kBK * 4;
-}
+size_t decode_gemm_smem_bytes(int NT, int N, int B, int64_t K) { return 1024 + gemm_smem(NT, N, B, K).total; }
 
 cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
                                cudaStream_t s) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
+  int dev = 0, smem_max = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  // the widest token tile (<= 256, a multiple of 16) whose stages fit
   int NT = (int)std::min<int64_t>(256, (T + 15) / 16 * 16);
+  while (NT > 16 && decode_gemm_smem_bytes(NT, d.N, d.bits, d.K) + 256 > (size_t)smem_max) NT -= 16;
+  if (decode_gemm_smem_bytes(NT, d.N, d.bits, d.K) + 256 > (size_t)smem_max) return cudaErrorNotSupported;
   CUtensorMap xmap;
   {
     cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)T};
@@ -347,12 +438,18 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   g.NT = NT;
   g.Y = Y;
   g.ldy = ldy;
-  const size_t smem = decode_gemm_smem_bytes(NT, d.N);
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(decode_gemm_kernel), smem);
-  if (e != cudaSuccess) return e;
+  const size_t smem = decode_gemm_smem_bytes(NT, d.N, d.bits, d.K);
   const dim3 grid((unsigned)((d.M + kBM - 1) / kBM), (unsigned)((T + NT - 1) / NT));
-  decode_gemm_kernel<<<grid, kThreads, smem, s>>>(xmap, g);
-  return cudaGetLastError();
+  // 11- and 10-bit codes with 128-column blocks compiled for their shape; anything else at run time
+  auto run = [&](auto kern) -> cudaError_t {
+    cudaError_t err = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, smem, s>>>(xmap, g);
+    return cudaGetLastError();
+  };
+  if (d.bits == 11 && d.log2b == 7) return run(decode_gemm_kernel<11, 7>);
+  if (d.bits == 10 && d.log2b == 7) return run(decode_gemm_kernel<10, 7>);
+  return run(decode_gemm_kernel<0, 0>);
 }
 
 }  // namespace qamw

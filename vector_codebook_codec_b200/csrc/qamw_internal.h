@@ -165,8 +165,9 @@ bool decode_tma_applicable(const DecodeArgs &a);
 cudaError_t launch_decode_tma(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_rotate_test(const RotateTestArgs &a, cudaStream_t s);
 // Decode fused with Y = X W_bf16^T on the tensor cores (qamw_decode_gemm.cu):
-// X bf16 [T][ldx], Y fp32 [T][ldy]; K % 128 == 0, b <= 128, N <= 2048.
-size_t decode_gemm_smem_bytes(int NT, int N);
+// X bf16 [T][ldx], Y fp32 [T][ldy]; K % 128 == 0, b <= 128, N <= 2048; cudaErrorNotSupported
+// if K is too wide for the shared-memory factor table.
+size_t decode_gemm_smem_bytes(int NT, int N, int B, int64_t K);
 cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
                                cudaStream_t s);
 // The same for b <= 512 with the 512-column rotation of the encode and calibrate kernels.
