@@ -1057,9 +1057,10 @@ def run_decode_gemm(args):
     Xs = {T: torch.from_numpy(synth.make_activations(T, K, 900 + T)).to(torch.bfloat16).to(dev) for T in DG_TOKENS}
     Ys = {T: torch.empty((T, M), dtype=torch.float32, device=dev) for T in DG_TOKENS}
     Wtmp = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    Ws = {T: torch.empty(q.decode_matmul_workspace_bytes(M, K, T), dtype=torch.uint8, device=dev) for T in DG_TOKENS}
 
     def fused(T):
-        q.decode_matmul(enc, Cd, Xs[T], status=status, out=Ys[T])
+        q.decode_matmul(enc, Cd, Xs[T], status=status, out=Ys[T], workspace=Ws[T])
 
     def unfused(T):
         q.decode(enc, Cd, out_dtype=torch.bfloat16, status=status, out=Wtmp)
@@ -1087,12 +1088,13 @@ def run_decode_gemm(args):
     torch.cuda.synchronize(dev)
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()} after warm-up")
-    # correctness at the smallest and largest T: fused vs unfused (same bf16 weights, fp32 accumulation)
+    # sanity at the smallest and largest T: fused vs decode to bf16 + matmul (the
+    # parity tests hold the derived bound against the oracle)
     for T in (DG_TOKENS[0], DG_TOKENS[-1]):
         fused(T)
         ref = torch.matmul(Xs[T].float(), Wb.float().T)
         scale = torch.matmul(Xs[T].float().abs(), Wb.float().abs().T)
-        if not bool(((Ys[T] - ref).abs() <= 2.0 ** -7 * scale + 1e-6).all()):
+        if not bool(((Ys[T] - ref).abs() <= 2.0 ** -6 * scale + 1e-6).all()):
             raise SystemExit(f"fused decode + matmul differs from decode + matmul at T={T}")
     clocks = ClockSampler(local)
     clocks.start()
@@ -1115,28 +1117,33 @@ def run_decode_gemm(args):
     tc_peak = float(peaks.get("bf16_tflops", 1590.0))
     wpr = q.words_per_row(K, spec.bits)
     t1 = rows[0]["fused_us"] * 1e-6
-    bytes1 = M * wpr * 4 + 4 * M + 4 * K + 2 * K + 8 * spec.N + 2 * K + 4 * M
+    # both kernels of the call at T = 1: packed words, r, codebook, Y; x (bf16),
+    # s, sigma, a (fp16, written then read), the token's power of two
+    bytes1 = M * wpr * 4 + 4 * M + 8 * spec.N + 4 * M + 2 * K + 4 * K + 2 * K + 2 * K + 2 * K + 8
     t4 = rows[-1]["fused_us"] * 1e-6
     flops4 = 2.0 * M * K * DG_TOKENS[-1]
     value = M * K / t1 / 1e9
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "Gweights/s", "n_gpus": 1, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; no checkpoint)",
+                "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded; no checkpoint)",
                 "config": {"workload": "decode_gemm_13824x5120_bf16_b128_N2048", "M": M, "K": K, "N": spec.N,
                            "bits": spec.bits, "tokens": list(DG_TOKENS),
-                           "op": "Y[T x M] = X[T x K] decode(W)^T, fp32 accumulation",
+                           "op": "Y[T x M] = X[T x K] decode(W)^T: decode's linear steps applied to X "
+                                 "(fp32, stored fp16 with a power of two per token), fp16 centroids, "
+                                 "fp32 accumulation on tcgen05",
                            "l2": "flushed by a 256 MiB write before every timed call",
                            "value_note": "weights per second of the fused call at T = 1"},
                 "roofline": {"bound": "hbm", "achieved": bytes1 / t1 / 1e9, "peak": hbm, "unit": "GB/s",
                              "frac": bytes1 / t1 / 1e9 / hbm, "traffic": None,
-                             "kernel": "decode_gemm_kernel at T = 1 (packed words, r, sigma, s, codebook, x, y)",
+                             "kernel": "prepare_x_kernel + decode_gemm_kernel at T = 1 (the whole call)",
                              "peak_source": f"{peak_kind} hbm_gbs"},
                 "rooflines": {"tensor_at_4096_tokens": {
                     "bound": "tensor", "achieved": flops4 / t4 / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
                     "frac": flops4 / t4 / 1e12 / tc_peak, "traffic": None,
-                    "kernel": "decode_gemm_kernel at T = 4096", "peak_source": f"{peak_kind} bf16_tflops (burst)"}},
-                "per_tokens": rows, "gpu_launches": len(DG_TOKENS) * 2 * max(args.steps, 3) + len(DG_TOKENS) * max(args.steps, 3),
+                    "kernel": "prepare_x_kernel + decode_gemm_kernel at T = 4096",
+                    "peak_source": f"{peak_kind} bf16_tflops (burst; fp16 runs at the bf16 rate)"}},
+                "per_tokens": rows, "gpu_launches": len(DG_TOKENS) * 3 * max(args.steps, 3),
                 "clocks": clk, "cpu_baseline": None, "e2e": None,
                 "timing": "each call timed alone with events after an L2 flush; median of the repetitions"}
         print(json.dumps(line), flush=True)

@@ -326,26 +326,45 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
 
 /*
  * qamw_decode_matmul -- Methodology (6) Decoding fused with the matrix
- * multiply that consumes the weights ("Significance and Claims": the decoded
- * weights are rounded to BF16 and fed to the matmul; the bit savings reach
- * latency once decoding is fused into it):
- *   Y[t][m] = sum_k X[t][k] * RN_bf16(w_hat[m][k])     (fp32 accumulation),
- * w_hat as qamw_decode computes it. The weights are decoded tile by tile into
- * shared memory and multiplied on the tensor cores (tcgen05, accumulators in
- * tensor memory); they are never written to device memory.
- *   packed, row_norm, sigma, col_scale, codebook: as qamw_decode
+ * multiply that consumes the weights ("Significance and Claims": the bit
+ * savings reach inference latency once decoding is fused into the matmul):
+ *   Y[t][m] = sum_j X[t][j] * w_hat[m][j],   w_hat as qamw_decode defines it,
+ * without forming w_hat. The decode's steps after the codebook lookup are
+ * linear and shared by all rows, and H_b is symmetric, so they are applied to
+ * the activations instead:
+ *   Y[t][m] = r_m * sum_i a_t[i] * C[idx(m, i/2)][i % 2],
+ *   a_t[i]  = sigma_{i/2} * (H_b (d (.) X[t] / s))_i / sqrt(b)   (per block of b columns).
+ * A first kernel computes a_t in fp32 and stores it in the workspace as fp16,
+ * scaled by a power of two 2^-e_t per token (its largest |a| lands in
+ * (2^13, 2^14]); a second streams the packed indices, looks up the centroids
+ * as fp16 pairs into the tensor-core operand tile in shared memory, multiplies
+ * on the tensor cores (tcgen05, fp32 accumulation in tensor memory) and
+ * scales by r_m 2^e_t. The weights never reach device memory.
+ * Accuracy: with S[t][m] = r_m sum_i |a_t[i] C[idx(m,i/2)][i%2]| and
+ * Q[t][m] = r_m sum_i sigma_{i/2} |C[..]| sum_{j in block(i)} |X[t][j] / s_j| / sqrt(b),
+ *   |Y - Y_exact| <= (2^-10 + K 2^-22) S + 2^-19 Q + (tiny fp16-subnormal terms),
+ * i.e. two fp16 roundings per product (2^-11 each) against the one bf16
+ * rounding (2^-8) of decoding to bf16 first.
+ *   packed, row_norm, sigma, col_scale, codebook: as qamw_decode (packed 8-byte, sigma 16-byte aligned)
  *   X : device bf16 [T][ldx] (activations, row-major; 16-byte aligned, ldx a multiple of 8)
- *   (packed must be 8-byte and sigma 16-byte aligned)
  *   Y : device float32 [T][ldy] (written for t < T, m < M)
- * Limits of this build: K a multiple of 128, block <= 128, N <= 2048
+ *   workspace : device, 256-byte aligned, >= qamw_decode_matmul_workspace_bytes(M, K, T)
+ *               bytes (the fp16 a_t, the per-token powers of two, and the partial sums
+ *               of output tiles whose K range is split between CTAs); owned by the caller
+ * Limits of this build: K a multiple of 128 and at most 32768
  * (QAMW_EUNSUPPORTED otherwise). Status bits as qamw_decode, plus
- * QAMW_STATUS_TIMEOUT if a bounded wait for a copy or a tensor-core result ran out.
- * Errors: QAMW_ENULL, QAMW_EINVAL (shape, T < 1, ldx / ldy, alignment), QAMW_EUNSUPPORTED.
+ * QAMW_STATUS_TIMEOUT if a bounded wait for a copy or a tensor-core result
+ * ran out. NaN or Inf activations propagate into Y as in any matrix product.
+ * Errors: QAMW_ENULL, QAMW_EINVAL (shape, T outside [1, 2^24], ldx / ldy,
+ * alignment, workspace too small), QAMW_EUNSUPPORTED.
  */
 int qamw_decode_matmul(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
                        int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
                        int32_t bits_per_pair, const void *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
-                       int32_t *status, qamw_stream_t stream);
+                       void *workspace, size_t workspace_bytes, int32_t *status, qamw_stream_t stream);
+/* Workspace bytes qamw_decode_matmul needs for M rows, K columns and T tokens
+ * (0 unless M, K >= 1 and 1 <= T <= 2^24). */
+size_t qamw_decode_matmul_workspace_bytes(int64_t M, int64_t K, int64_t T);
 
 /*
  * qamw_rotate_rows -- the rotation alone, for tests of step (2).

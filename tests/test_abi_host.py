@@ -235,3 +235,31 @@ def test_encode_prepared_rejects_on_host(lib):
                dict(table=ctypes.c_void_p(0x10008))):
         assert call(**kw) == QAMW_EINVAL
     assert call(N=16384, bits=16) == QAMW_EUNSUPPORTED
+
+
+def test_decode_matmul_rejects_on_host(lib):
+    ws = lib.qamw_decode_matmul_workspace_bytes(128, 256, 16)
+    assert ws >= 16 * 256 * 2 + 16 * 4 and ws % 256 == 0
+    assert lib.qamw_decode_matmul_workspace_bytes(128, 256, 0) == 0
+    assert lib.qamw_decode_matmul_workspace_bytes(0, 256, 16) == 0
+    assert lib.qamw_decode_matmul_workspace_bytes(128, 256, (1 << 24) + 1) == 0
+
+    def call(**kw):
+        a = dict(packed=FAKE, r=FAKE, sigma=FAKE, s=None, M=128, K=256, block=128, seed=1, cb=FAKE, N=2048,
+                 bits=11, X=FAKE, T=16, ldx=256, Y=FAKE, ldy=128, ws=FAKE, nws=ws, status=None, stream=None)
+        a.update(kw)
+        return lib.qamw_decode_matmul(a["packed"], a["r"], a["sigma"], a["s"], a["M"], a["K"], a["block"],
+                                      a["seed"], a["cb"], a["N"], a["bits"], a["X"], a["T"], a["ldx"], a["Y"],
+                                      a["ldy"], a["ws"], a["nws"], a["status"], a["stream"])
+    for kw in (dict(packed=None), dict(r=None), dict(sigma=None), dict(cb=None), dict(X=None), dict(Y=None),
+               dict(ws=None)):
+        assert call(**kw) == QAMW_ENULL
+    for kw in (dict(T=0), dict(T=(1 << 24) + 1), dict(ldx=255), dict(ldy=127), dict(X=ctypes.c_void_p(0x10008)), dict(ldx=260),
+               dict(packed=ctypes.c_void_p(0x10004)), dict(sigma=ctypes.c_void_p(0x10008)),
+               dict(ws=ctypes.c_void_p(0x10080)), dict(nws=ws - 1),
+               dict(block=96), dict(N=2049)):
+        assert call(**kw) == QAMW_EINVAL
+    assert call(K=384 - 128 + 64, ldx=384) == QAMW_EINVAL               # K = 320: not a multiple of the block
+    assert call(K=192, block=64, ldx=192) == QAMW_EUNSUPPORTED          # K not a multiple of 128
+    big = lib.qamw_decode_matmul_workspace_bytes(128, 32768 + 128, 16)
+    assert call(K=32768 + 128, ldx=32768 + 128, nws=big) == QAMW_EUNSUPPORTED

@@ -55,7 +55,8 @@ _SIGNATURES = {
     "qamw_rotate_rows": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_i32, _c_p]),
     "qamw_search_cells": (ctypes.c_int, [_c_p, _c_i64, _c_p, _c_p, _c_p]),
     "qamw_decode_matmul": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _c_u64, _c_p, _c_i32,
-                                          _c_i32, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_p]),
+                                          _c_i32, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_sz, _c_p, _c_p]),
+    "qamw_decode_matmul_workspace_bytes": (_c_sz, [_c_i64, _c_i64, _c_i64]),
     "qamw_encode_prepared": (ctypes.c_int, [_c_p, ctypes.c_int, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i32, _c_u64,
                                             _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_p, _c_p, _c_p]),
     "qamw_search_table_bytes": (_c_sz, [_c_i32]),
@@ -139,6 +140,10 @@ qamw_lloyd_train = _raw("qamw_lloyd_train")
 qamw_calibrate_sigma_noalloc = _raw("qamw_calibrate_sigma_noalloc")
 qamw_search_table_bytes = _raw("qamw_search_table_bytes")
 qamw_build_search_table = _raw("qamw_build_search_table")
+qamw_encode_prepared = _raw("qamw_encode_prepared")
+qamw_search_cells = _raw("qamw_search_cells")
+qamw_decode_matmul = _raw("qamw_decode_matmul")
+qamw_decode_matmul_workspace_bytes = _raw("qamw_decode_matmul_workspace_bytes")
 
 
 # ---------------------------------------------------------------------------
@@ -443,9 +448,15 @@ def decode(enc: Encoded, codebook, out_dtype=None, status=None, stream=None, out
     return out
 
 
-def decode_matmul(enc: Encoded, codebook, X, status=None, stream=None, out=None):
-    """Y = X @ RN_bf16(decode(enc))^T with the decode fused into the tensor-core
-    matmul (qamw_decode_matmul); X is a bf16 CUDA tensor [T, K], Y float32 [T, M]."""
+def decode_matmul_workspace_bytes(M: int, K: int, T: int) -> int:
+    return int(load_library().qamw_decode_matmul_workspace_bytes(M, K, T))
+
+
+def decode_matmul(enc: Encoded, codebook, X, status=None, stream=None, out=None, workspace=None):
+    """Y = X @ decode(enc)^T with the decode fused into the tensor-core matmul
+    (qamw_decode_matmul); X is a bf16 CUDA tensor [T, K], Y float32 [T, M].
+    ``workspace`` (a CUDA uint8 tensor of decode_matmul_workspace_bytes(M, K, T)
+    bytes) is allocated here when not given."""
     torch = _torch()
     _need_cuda("codebook", codebook, torch.float32, 2)
     _need_cuda("X", X, torch.bfloat16, 2)
@@ -453,10 +464,14 @@ def decode_matmul(enc: Encoded, codebook, X, status=None, stream=None, out=None)
         raise ValueError("X must have K columns")
     T = X.shape[0]
     Y = torch.empty((T, enc.M), dtype=torch.float32, device=X.device) if out is None else out
+    nws = decode_matmul_workspace_bytes(enc.M, enc.K, T)
+    if workspace is None:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=X.device)
     _check("qamw_decode_matmul", load_library().qamw_decode_matmul(
         _ptr(enc.packed), _ptr(enc.row_norm), _ptr(enc.sigma), _ptr(enc.col_scale), enc.M, enc.K, enc.block,
         enc.seed & (2**64 - 1), _ptr(codebook.contiguous()), codebook.shape[0], enc.bits, _ptr(X), T, _ld(X),
-        _ptr(Y), _ld(Y), _ptr(status), _stream_ptr(stream)))
+        _ptr(Y), _ld(Y), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream_ptr(stream)))
     return Y
 
 

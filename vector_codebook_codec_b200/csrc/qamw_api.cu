@@ -406,24 +406,27 @@ int qamw_encode_polar(const void *W, qamw_dtype w_dtype, int64_t M, int64_t K, i
 int qamw_decode_matmul(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,
                        int64_t M, int64_t K, int32_t block, uint64_t sign_seed, const float *codebook, int32_t N,
                        int32_t bits_per_pair, const void *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
-                       int32_t *status, qamw_stream_t stream) {
+                       void *workspace, size_t workspace_bytes, int32_t *status, qamw_stream_t stream) {
   static const char *fn = "qamw_decode_matmul";
   CallRange nvtx_range(fn);
   g_last_error[0] = 0;
   int rc;
-  if (!packed || !row_norm || !sigma || !codebook || !X || !Y)
-    return fail(QAMW_ENULL, "%s: packed, row_norm, sigma, codebook, X and Y must be non-NULL", fn);
+  if (!packed || !row_norm || !sigma || !codebook || !X || !Y || !workspace)
+    return fail(QAMW_ENULL, "%s: packed, row_norm, sigma, codebook, X, Y and workspace must be non-NULL", fn);
   if ((rc = check_shape(M, K, block, fn))) return rc;
   if ((rc = check_code(N, bits_per_pair, fn))) return rc;
-  if (T < 1) return fail(QAMW_EINVAL, "%s: T (%lld) must be >= 1", fn, (long long)T);
+  if (T < 1 || T > (int64_t)1 << 24) return fail(QAMW_EINVAL, "%s: T (%lld) must be in [1, 2^24]", fn, (long long)T);
   if (ldx < K || ldy < M)
     return fail(QAMW_EINVAL, "%s: ldx (%lld) must be >= K and ldy (%lld) >= M", fn, (long long)ldx, (long long)ldy);
-  if (K % 128 != 0 || block > 128 || N > 2048 || T > (int64_t)1 << 30)
-    return fail(QAMW_EUNSUPPORTED, "%s: needs K a multiple of 128, block <= 128, N <= 2048, T <= 2^30", fn);
+  if (K % 128 != 0 || K > 32768)
+    return fail(QAMW_EUNSUPPORTED, "%s: needs K a multiple of 128 and at most 32768", fn);
   if (reinterpret_cast<uintptr_t>(X) % 16 != 0 || ldx % 8 != 0)
     return fail(QAMW_EINVAL, "%s: X must be 16-byte aligned with ldx a multiple of 8", fn);
   if (reinterpret_cast<uintptr_t>(packed) % 8 != 0 || reinterpret_cast<uintptr_t>(sigma) % 16 != 0)
     return fail(QAMW_EINVAL, "%s: packed must be 8-byte and sigma 16-byte aligned", fn);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 || workspace_bytes < decode_matmul_workspace_bytes(M, K, T))
+    return fail(QAMW_EINVAL, "%s: workspace must be 256-byte aligned and hold %zu bytes (got %zu)", fn,
+                decode_matmul_workspace_bytes(M, K, T), workspace_bytes);
   DecodeArgs a;
   a.packed = packed;
   a.row_norm = row_norm;
@@ -441,8 +444,14 @@ int qamw_decode_matmul(const uint32_t *packed, const float *row_norm, const floa
   a.out_t = QAMW_BF16;
   a.ldo = 0;
   a.status = status;
-  cudaError_t e = launch_decode_gemm(a, static_cast<const uint16_t *>(X), T, ldx, Y, ldy, (cudaStream_t)stream);
+  cudaError_t e = launch_decode_gemm(a, static_cast<const uint16_t *>(X), T, ldx, Y, ldy, workspace,
+                                     (cudaStream_t)stream);
   return e == cudaSuccess ? QAMW_OK : cuda_fail(e, fn);
+}
+
+size_t qamw_decode_matmul_workspace_bytes(int64_t M, int64_t K, int64_t T) {
+  if (M < 1 || K < 1 || T < 1 || T > (int64_t)1 << 24) return 0;
+  return decode_matmul_workspace_bytes(M, K, T);
 }
 
 int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigma, const float *col_scale,

@@ -2,29 +2,53 @@
 // consumes the weights, on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // "QAM-W: Joint 2D Codebook Quantization for LLM Weights ...", Methodology (6)
-// Decoding, and "Significance and Claims": the decoded weights are rounded to
-// BF16 and fed to the matrix multiply; the bit savings reach latency only
-// with a fused kernel. Here
-//   Y[t][m] = sum_k X[t][k] * W_bf16[m][k],   W_bf16 = RN_bf16(w_hat),
-//   w_hat[m][j] = r_m * d_j * (H_b (sigma (.) C[idx]))_j / (sqrt(b) s_j),
-// with the weights never leaving the chip: each CTA owns 128 output rows
-// (features) and one tile of NT tokens, and walks K in chunks of 128 columns.
-// For every chunk its 8 warps unpack the chunk's indices, look up and rescale
-// the centroids, apply the inverse Hadamard butterflies in fp32 (block bits
-// 0..4 in registers, 5..6 across the 4 lanes of a row), scale by r_m d_j /
-// (sqrt(b) s_j) and write the bf16 tile into shared memory in the 128-byte
-// swizzled K-major layout of the tensor cores; one TMA tensor copy (no
-// multicast) brings the matching X tile in the same layout. One thread then
-// issues the chunk's eight 128 x NT x 16 tcgen05.mma (bf16 in, fp32
-// accumulated in tensor memory) and commits them to an mbarrier; the next
-// chunk is decoded into the other stage meanwhile. At the end the accumulator
-// is read from tensor memory (tcgen05.ld) and written as fp32 Y.
+// Decoding, and "Significance and Claims" (the bit savings reach inference
+// latency only once decoding is fused into the matrix multiply). The product
+//   Y[t][m] = sum_j X[t][j] w_hat[m][j],
+//   w_hat[m][j] = r_m d_j (H_b y_m)_j / (sqrt(b) s_j),  y_m[2k+e] = sigma_k C[idx(m,k)][e],
+// is formed without w_hat. Every decode step after the codebook lookup is
+// linear and the same for all rows, and H_b is symmetric, so those steps move
+// to the activations:
+//   Y[t][m] = r_m sum_i a_t[i] C[idx(m, i/2)][i%2],
+//   a_t[i]  = sigma_{i/2} (H_b (d (.) X[t] / s))_i / sqrt(b)      (per block of b columns),
+// which costs log2 b adds per activation instead of per weight.
 //
-// Every wait (TMA arrival, MMA completion) is a bounded mbarrier wait; a wait
-// that runs out sets QAMW_STATUS_TIMEOUT and the CTA stops, frees its tensor
-// memory and returns.
+// Kernel 1 (prepare_x_kernel): a cluster of up to 8 CTAs per token computes
+// a_t in fp32 (each CTA a share of the columns), agrees on the token's
+// largest |a| through distributed shared memory, scales by 2^-e_t so that it
+// lies in (2^13, 2^14], and stores fp16 a_t and 2^e_t. It also clears the
+// tile counters of kernel 2.
+//
+// Kernel 2 (decode_gemm_kernel), persistent: one CTA per SM. The work is the
+// list of (output tile, K chunk) units -- an output tile is 128 rows m x NT
+// tokens, a chunk 128 columns (64 pairs) -- split into equal contiguous
+// ranges, one per CTA ("stream-K"), so every SM gets the same number of
+// chunks whatever the number of tiles. Warp roles:
+//   warps 0-15  unpack the chunk's indices of the 128 rows, look the centroids
+//               up as fp16 pairs and write the 128 x 128 operand tile into
+//               shared memory in the tensor cores' swizzled K-major layout;
+//   warp 16     streams the packed indices into a ring of word stages (one TMA
+//               tensor copy per chunk, or cp.async when the row pitch is not a
+//               multiple of 16 bytes);
+//   warp 17     streams the fp16 a tile of the chunk (TMA, 128-byte swizzle);
+//   warp 18     issues the chunk's eight 128 x NT x 16 tcgen05.mma (fp16 in,
+//               fp32 accumulated in tensor memory, two accumulators used in
+//               turn) and commits them to mbarriers;
+//   warps 19-22 read a finished accumulator (tcgen05.ld) and write
+//               Y = r_m 2^e_t acc; a tile whose chunks were split between CTAs
+//               is written as partial sums to the workspace, and the CTA that
+//               finishes it last adds the parts in a fixed order.
+// Stages hand over through mbarriers (full / empty per stage), so the roles
+// run ahead of one another by up to the ring depth; no CTA-wide barrier sits
+// in the loop.
+//
+// Every wait is a bounded mbarrier wait; one that runs out sets
+// QAMW_STATUS_TIMEOUT, the other roles see the CTA's failure flag and stop,
+// the copies and MMAs already in flight are waited for (again bounded), the
+// tensor memory is freed and the kernel returns.
 #include <algorithm>
 #include <cmath>
+#include <cuda_fp16.h>
 
 #include "qamw_device.cuh"
 #include "qamw_internal.h"
@@ -34,40 +58,83 @@
 namespace qamw {
 namespace {
 
-constexpr int kBM = 128;              // output rows per CTA (tensor-memory lanes)
-constexpr int kBK = 128;              // columns per chunk (whole Hadamard blocks, b <= 128)
-constexpr int kWarps = 16;            // one (row, 32-column quarter) of the chunk per thread
-constexpr int kThreads = kWarps * 32;
-constexpr int kAtomBytesA = kBM * 128;                // one 64-column swizzle atom of the weight tile
-constexpr int kStageBytesA = 2 * kAtomBytesA;         // 128 columns = 2 atoms
-constexpr uint32_t kWaitLimit = 1u << 22;             // mbarrier try_wait attempts
+constexpr int kBM = 128;                   // output rows per tile (tensor-memory lanes)
+constexpr int kBK = 128;                   // columns (64 pairs) per chunk
+constexpr int kDecWarps = 16;              // thread: row 8 w + lane / 4, pairs 16 (lane % 4) .. + 15
+constexpr int kWarpWords = kDecWarps;      // streams the packed words
+constexpr int kWarpX = kDecWarps + 1;      // streams the activation tiles
+constexpr int kWarpMma = kDecWarps + 2;    // issues the MMAs
+constexpr int kWarpEpi = kDecWarps + 3;    // first of the 4 epilogue warps
+constexpr int kThreads = (kDecWarps + 7) * 32;
+constexpr int kAtomBytes = kBM * 128;      // one 64-column swizzle atom of the 128-row operand tile
+constexpr int kStageBytesA = 2 * kAtomBytes;
+constexpr int kMaxStages = 8;
+constexpr int kMaxCtas = 160;              // persistent CTAs at most (the partial-sum slots are sized for it)
+constexpr uint32_t kWaitTries = 1u << 22;  // try_wait attempts before a spinning wait gives up
+constexpr uint32_t kSleepTries = 1u << 21; // attempts (<= 512 ns apart) before a sleeping wait gives up
+constexpr int kPrepThreads = 128;          // small enough to share an SM with a CTA of kernel 2
+constexpr int kPrepSmemReserve = 18 * 1024;   // shared memory kernel 2 leaves to one CTA of kernel 1
+constexpr int kPrepCluster = 8;            // CTAs per token in kernel 1 (portable cluster size)
+
+// ---------------------------------------------------------------------------
+// workspace: [a: T x K fp16][2^e_t: T fp32][tile counters][partial sums]
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+__host__ __device__ __forceinline__ int nt_cap(int64_t T) { return (int)(T >= 256 ? 256 : (T + 15) / 16 * 16); }
+struct WsLayout {
+  size_t off_scale, off_cnt, off_part, total;
+};
+__host__ __device__ __forceinline__ WsLayout ws_layout(int64_t M, int64_t K, int64_t T) {
+  WsLayout w;
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((T + 15) / 16);   // tiles for the narrowest token tile
+  w.off_scale = align256((size_t)T * (size_t)K * 2);
+  w.off_cnt = w.off_scale + align256((size_t)T * 4);
+  w.off_part = w.off_cnt + align256((size_t)tiles * 4);
+  w.total = w.off_part + (size_t)2 * kMaxCtas * (size_t)nt_cap(T) * kBM * 4;
+  return w;
+}
 
 struct GemmArgs {
-  DecodeArgs d;          // packed, row_norm, sigma, col_scale, M, K, log2b, seed, codebook, N, bits, wpr, status
-  int64_t T;             // tokens
-  int NT;                // tokens per CTA tile (16..256, multiple of 16)
-  float *Y;              // [T][ldy] fp32
-  int64_t ldy;
+  const uint32_t *packed;   // [M][wpr]
+  const float *row_norm;    // [M]
+  const float *codebook;    // [N][2] fp32
+  const float *tok_scale;   // [T] 2^e_t
+  uint32_t *counters;       // [tiles] contributions received (cleared by kernel 1)
+  float *part;              // [2 * CTAs][NT][128] partial sums
+  float *Y;                 // [T][ldy]
+  int64_t ldy, M, K, T, wpr;
+  int64_t n_m;              // row tiles
+  int64_t n_units;          // tiles x chunks
+  int N, bits;
+  int NT;                   // tokens per tile (16..256, a multiple of 16)
+  int SA;                   // operand stages (weight tile + activation tile)
+  int SW;                   // word stages
+  int BW;                   // staged words per row and chunk
+  int words_tma;            // 1: words by TMA; 0: by cp.async
+  int32_t *status;
 };
 
-// shared-memory layout after the 1024-aligned operand stages
+// shared-memory layout (after 1024-byte alignment): SA weight tiles, SA
+// activation tiles, SW word stages, the fp16 codebook
 struct GemmSmem {
-  int stage_b, words_row, words_stage;
-  size_t off_b, off_words, off_cb, off_fac, off_sig, total;
+  int stage_x, wpitch;
+  size_t off_x, off_w, off_cb, total;
 };
-constexpr int kWordStages = 3;   // packed words of a chunk are fetched two chunks ahead
-__host__ __device__ __forceinline__ GemmSmem gemm_smem(int NT, int N, int B, int64_t K) {
+__host__ __device__ __forceinline__ GemmSmem gemm_smem(int NT, int SA, int SW, int BW, int N) {
   GemmSmem g;
-  g.stage_b = NT * 256;                          // 2 atoms of NT rows x 128 B
-  g.words_row = 2 * B;                           // a row's packed words of one chunk (64 pairs)
-  g.words_stage = kBM * g.words_row + 4;         // + 4: the unpacking reads one word past a row
-  g.off_b = 2 * (size_t)kStageBytesA;
-  g.off_words = g.off_b + 2 * (size_t)g.stage_b;
-  g.off_cb = g.off_words + kWordStages * (size_t)g.words_stage * 4;
-  g.off_fac = (g.off_cb + (size_t)N * 8 + 15) & ~(size_t)15;   // 16-byte loads of the factors
-  g.off_sig = g.off_fac + (size_t)K * 4;                        // every column's factor, computed once
-  g.total = g.off_sig + kWordStages * (kBK / 2) * 4;
+  g.stage_x = NT * 256;                                  // 2 atoms of NT rows x 128 B
+  g.wpitch = (kBM * BW * 4 + 16 + 127) & ~127;           // + 16: the unpacking reads past the last row
+  g.off_x = (size_t)SA * kStageBytesA;
+  g.off_w = g.off_x + (size_t)SA * g.stage_x;
+  g.off_cb = g.off_w + (size_t)SW * g.wpitch;
+  g.total = g.off_cb + (size_t)N * 4;
   return g;
+}
+
+// the contiguous unit range [u0, u1) of CTA b of G, and the CTA holding unit u
+__host__ __device__ __forceinline__ int64_t range_start(int64_t b, int64_t G, int64_t total) { return b * total / G; }
+__host__ __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t G, int64_t total) {
+  return ((u + 1) * G - 1) / total;
 }
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
@@ -80,6 +147,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }   // the 4 epilogue warps
+// barrier of the 4 epilogue warps that returns whether any of their threads passed true
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile("{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, 1, 128, p; selp.u32 %0, 1, 0, q; }"
+               : "=r"(r)
+               : "r"((uint32_t)v)
+               : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// arrive once all of this thread's earlier cp.async copies have landed (the
+// barrier's expected count includes this arrival)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// programmatic dependent launch: kernel 2 starts while kernel 1 runs, and
+// waits for kernel 1's results only where it reads them
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
   asm volatile(
@@ -89,8 +179,8 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -116,6 +206,51 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// Bounded waits that also give up once another role of the CTA has failed:
+// 0 = the phase completed, 1 = the CTA failed elsewhere, 2 = this wait ran out
+// (it then raises the CTA's failure flag). wait_phase spins (the pipeline's
+// hand-overs); wait_phase_sleep backs off with nanosleep (the epilogue's wait
+// for a whole tile), leaving the issue slots to the decode warps.
+__device__ __forceinline__ int wait_phase(uint64_t *bar, uint32_t parity, volatile int *fail) {
+  for (uint32_t i = 0; i < kWaitTries; ++i) {
+    if (mbar_try_wait(bar, parity)) return 0;
+    if ((i & 63u) == 63u && *fail) return 1;
+  }
+  *fail = 1;
+  return 2;
+}
+__device__ __forceinline__ int wait_phase_sleep(uint64_t *bar, uint32_t parity, volatile int *fail) {
+  uint32_t ns = 32;
+  for (uint32_t i = 0; i < kSleepTries; ++i) {
+    if (mbar_try_wait(bar, parity)) return 0;
+    if (*fail) return 1;
+    __nanosleep(ns);
+    if (ns < 512) ns <<= 1;
+  }
+  *fail = 1;
+  return 2;
+}
+
+// position of a unit: tile = mt + n_m tt (row tile mt, token tile tt), chunk c;
+// walked incrementally (no 64-bit division per unit)
+struct Cursor {
+  int64_t tile, mt, tt;
+  int c;
+  __device__ __forceinline__ Cursor(int64_t u, int n_chunks, int64_t n_m) {
+    tile = u / n_chunks;
+    c = (int)(u - tile * n_chunks);
+    tt = tile / n_m;
+    mt = tile - tt * n_m;
+  }
+  __device__ __forceinline__ void next(int n_chunks, int64_t n_m) {
+    if (++c == n_chunks) {
+      c = 0;
+      ++tile;
+      if (++mt == n_m) { mt = 0; ++tt; }
+    }
+  }
+};
 
 // The 16 indices of pairs 16 q .. 16 q + 15 of a row's chunk, from its 2B
 // staged words (LSB-first B-bit fields). BB > 0: B fixed at compile time (the
@@ -152,75 +287,250 @@ __device__ __forceinline__ void unpack16(const uint32_t *rw, int q, int B, uint3
   }
 }
 
-// BB > 0 fixes the code size, LB > 0 log2 b, at compile time (a butterfly
-// stage guarded by a run-time block size costs register copies where the two
-// paths join); 0 reads them at run time.
-template <int BB, int LB>
-__global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs g) {
+// ----------------------------------------------------------------------------
+// Kernel 1: a_t = sigma (.) H_b (d (.) x_t / s) / sqrt(b), fp16 with 2^e_t.
+// Cluster of S CTAs per token (blocks S t .. S t + S - 1); CTA rank c takes the column units
+// c, c + S, ... (a unit is 512 columns, or one block when b = 1024) and keeps
+// them in shared memory as fp32.
+// ----------------------------------------------------------------------------
+struct PrepArgs {
+  const uint16_t *X;        // bf16 [T][ldx]
+  int64_t ldx, T, K;
+  const float *sigma;       // [K/2]
+  const float *col_scale;   // [K] or nullptr
+  uint64_t seed;
+  int log2b;
+  int S;                    // CTAs per token (cluster size)
+  __half *A;                // fp16 [T][K]
+  float *tok_scale;         // [T]
+  uint32_t *counters;       // cleared here
+  int64_t n_counters;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// at most 48 registers: one CTA fits beside a CTA of kernel 2 (736 threads x 80 registers)
+__global__ void __launch_bounds__(kPrepThreads, 10) prepare_x_kernel(PrepArgs p) {
+  extern __shared__ __align__(16) float vloc[];   // the CTA's units, fp32, one after the other
+  __shared__ float red[kPrepThreads / 32];
+  __shared__ float cta_max;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.S;
+  const int64_t t = blockIdx.x / S;
+  const int64_t K = p.K;
+  const int lb = p.log2b;
+  const int rank = (int)cluster_rank();
+  const int ucols = lb > 9 ? (1 << lb) : 512;       // columns per unit
+  const int64_t n_units = (K + ucols - 1) / ucols;
+  const int64_t n_mine = n_units > rank ? (n_units - rank + S - 1) / S : 0;
+  const int lreg = lb < 4 ? lb : 4, lshf = lb < 9 ? lb : 9;
+  const uint16_t *xr = p.X + t * p.ldx;
+
+  griddep_launch_dependents();
+  if (t == 0 && rank == 0)
+    for (int64_t i = threadIdx.x; i < p.n_counters; i += kPrepThreads) p.counters[i] = 0u;
+  const float inv_sqrt_b = (float)(1.0 / sqrt((double)(1 << lb)));
+  float mx = 0.0f;   // the largest |a| of the CTA's columns
+
+  // block bits 0..3 in registers (16 consecutive columns per lane), 4..8
+  // across the lanes of a warp (a 512-column span per warp), 9 in shared memory
+  const int64_t n_spans = n_mine * (ucols / 512);
+  for (int64_t sp = warp; sp < n_spans; sp += kPrepThreads / 32) {
+    const int64_t li = sp / (ucols / 512), part = sp % (ucols / 512);
+    const int64_t col = (rank + li * S) * (int64_t)ucols + part * 512 + 16 * lane;
+    float *dst = vloc + li * ucols + part * 512 + 16 * lane;
+    const bool in = col < K;   // K % 16 == 0: a lane's 16 columns are all in or all out
+    float u[16];
+    if (in) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(xr + col);
+      const uint4 q0 = src[0], q1 = src[1];
+      const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float x = __uint_as_float(((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu)) << 16);
+        float v = p.col_scale != nullptr ? __fdiv_rn(x, p.col_scale[col + e]) : x;
+        if (mask_is_negative(p.seed, col + e)) v = -v;
+        u[e] = v;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) u[e] = 0.0f;
+    }
+#pragma unroll
+    for (int tb = 0; tb < 4; ++tb) {
+      if (tb < lreg) {
+        const int h = 1 << tb;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          if ((e & h) == 0) {
+            const float a0 = u[e], a1 = u[e | h];
+            u[e] = a0 + a1;
+            u[e | h] = a0 - a1;
+          }
+        }
+      }
+    }
+    for (int tb = 4; tb < lshf; ++tb) {   // warp-uniform
+      const int h = 1 << (tb - 4);
+      const float sgn = (lane & h) ? -1.0f : 1.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) u[e] = __fmaf_rn(sgn, u[e], __shfl_xor_sync(0xffffffffu, u[e], h));
+    }
+    if (lb <= 9 && in) {   // every butterfly done: times sigma_k / sqrt(b) here
+      const float4 *sg = reinterpret_cast<const float4 *>(p.sigma + (col >> 1));   // col % 16 == 0: 32-byte aligned
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float4 s4 = sg[h];
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float gk = __fmul_rn(sv[k], inv_sqrt_b);
+          u[8 * h + 2 * k] = __fmul_rn(u[8 * h + 2 * k], gk);
+          u[8 * h + 2 * k + 1] = __fmul_rn(u[8 * h + 2 * k + 1], gk);
+          mx = fmaxf(mx, fmaxf(fabsf(u[8 * h + 2 * k]), fabsf(u[8 * h + 2 * k + 1])));
+        }
+      }
+    }
+    float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d4[i] = make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+  }
+  __syncthreads();
+  const int64_t n_loc = n_mine * ucols;
+  if (lb > 9) {   // b = 1024: bit 9 pairs the two halves of every unit, then sigma_k / sqrt(b)
+    const int h = 512;
+    for (int64_t i = threadIdx.x; i < n_mine * h; i += kPrepThreads) {
+      const int64_t li = i / h, o = i % h;
+      float *v = vloc + li * ucols + o;
+      const float a0 = v[0], a1 = v[h];
+      v[0] = a0 + a1;
+      v[h] = a0 - a1;
+    }
+    __syncthreads();
+    for (int64_t i = 2 * threadIdx.x; i < n_loc; i += 2 * kPrepThreads) {
+      const int64_t li = i / ucols, o = i % ucols;
+      const int64_t col = (rank + li * S) * (int64_t)ucols + o;   // K % 1024 == 0: always < K
+      const float gk = __fmul_rn(p.sigma[col >> 1], inv_sqrt_b);
+      float2 v = *reinterpret_cast<float2 *>(vloc + i);
+      v.x = __fmul_rn(v.x, gk);
+      v.y = __fmul_rn(v.y, gk);
+      *reinterpret_cast<float2 *>(vloc + i) = v;
+      mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int w = 1; w < kPrepThreads / 32; ++w) m = fmaxf(m, red[w]);
+    cta_max = m;
+  }
+  cluster_sync();   // every CTA of the token has published its largest |a|
+  if (warp == 0) {
+    float m = lane < S ? ld_cluster_f32(&cta_max, (uint32_t)lane) : 0.0f;
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[0] = m;
+  }
+  __syncthreads();
+  mx = red[0];
+  // e = ceil(log2 mx) - 14, so that mx 2^-e lies in (2^13, 2^14]; 0 for a zero
+  // or non-finite token (the latter then propagates into Y as in any product)
+  int e = 0;
+  if (mx > 0.0f && mx <= 3.0e38f) {
+    int ex;
+    const float fr = frexpf(mx, &ex);   // mx = fr 2^ex, fr in [0.5, 1)
+    e = (fr == 0.5f ? ex - 1 : ex) - 14;
+    e = max(-112, min(112, e));
+  }
+  const float down = __int_as_float((127 - e) << 23);   // 2^-e, exact
+  if (rank == 0 && threadIdx.x == 0) p.tok_scale[t] = __int_as_float((127 + e) << 23);
+  __half *ar = p.A + t * K;
+  for (int64_t i = 8 * (int64_t)threadIdx.x; i < n_loc; i += 8 * kPrepThreads) {
+    const int64_t li = i / ucols, o = i % ucols;
+    const int64_t col = (rank + li * S) * (int64_t)ucols + o;
+    if (col >= K) continue;
+    const float4 v0 = *reinterpret_cast<const float4 *>(vloc + i), v1 = *reinterpret_cast<const float4 *>(vloc + i + 4);
+    const __half2 h0 = __floats2half2_rn(v0.x * down, v0.y * down), h1 = __floats2half2_rn(v0.z * down, v0.w * down);
+    const __half2 h2 = __floats2half2_rn(v1.x * down, v1.y * down), h3 = __floats2half2_rn(v1.z * down, v1.w * down);
+    uint4 o4;
+    o4.x = *reinterpret_cast<const uint32_t *>(&h0);
+    o4.y = *reinterpret_cast<const uint32_t *>(&h1);
+    o4.z = *reinterpret_cast<const uint32_t *>(&h2);
+    o4.w = *reinterpret_cast<const uint32_t *>(&h3);
+    *reinterpret_cast<uint4 *>(ar + col) = o4;
+  }
+  cluster_sync();   // no CTA leaves while another may still read its cta_max
+}
+
+// ----------------------------------------------------------------------------
+// Kernel 2: unpack + lookup into the operand tile, tcgen05 MMA, epilogue.
+// ----------------------------------------------------------------------------
+template <int BB>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap, GemmArgs g) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   // 1024-byte alignment for the swizzled operand tiles
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const DecodeArgs &a = g.d;
-  const int NT = g.NT;
-  const int B = BB > 0 ? BB : a.bits;
-  const GemmSmem L = gemm_smem(NT, a.N, B, a.K);
-  unsigned char *A0 = smem;                                          // [2][kStageBytesA]
-  unsigned char *B0 = smem + L.off_b;                                // [2][stage_b]
-  uint32_t *W0 = reinterpret_cast<uint32_t *>(smem + L.off_words);   // [2][words_stage] packed words of a chunk
-  float2 *cbf = reinterpret_cast<float2 *>(smem + L.off_cb);         // (c0 + c1, c0 - c1): the first butterfly folded in
-  float *fac = reinterpret_cast<float *>(smem + L.off_fac);          // [K] d_j / (sqrt(b) s_j)
-  float *S0 = reinterpret_cast<float *>(smem + L.off_sig);           // [kWordStages][64] sigma of a chunk
+  const int B = BB > 0 ? BB : g.bits;
+  const int NT = g.NT, SA = g.SA, SW = g.SW;
+  const GemmSmem L = gemm_smem(NT, SA, SW, g.BW, g.N);
+  unsigned char *A0 = smem;                                          // [SA][kStageBytesA]
+  unsigned char *X0 = smem + L.off_x;                                // [SA][stage_x]
+  unsigned char *W0 = smem + L.off_w;                                // [SW][wpitch]
+  uint32_t *cb = reinterpret_cast<uint32_t *>(smem + L.off_cb);      // [N] fp16 pairs
 
-  __shared__ __align__(8) uint64_t bar_x[2], bar_mma[2];
+  __shared__ __align__(8) uint64_t full_w[kMaxStages], empty_w[kMaxStages];
+  __shared__ __align__(8) uint64_t full_x[kMaxStages], full_a[kMaxStages], empty_a[kMaxStages];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
+  __shared__ int s_last;
+  volatile int *fail = &s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * kBM;
-  const int64_t t0 = (int64_t)blockIdx.y * NT;
-  const int64_t n_chunks = a.K / kBK;
-  const int log2b = LB > 0 ? LB : a.log2b;
-  const float inv_sqrt_b = (float)(1.0 / sqrt((double)(1 << log2b)));
-  const uint32_t tmem_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
+  const int n_chunks = (int)(g.K / kBK);
+  const int64_t G = gridDim.x;
+  const int64_t u0 = range_start(blockIdx.x, G, g.n_units), u1 = range_start(blockIdx.x + 1, G, g.n_units);
+  const uint32_t acc_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
+  const uint32_t tmem_cols = 2 * acc_cols;
 
-  // packed words and sigma of chunk c into staging buffer c % 3 (cp.async, 8 bytes
-  // at a time: a row's 2B words of a chunk start 8B-byte aligned; four threads
-  // per row; rows past M read as 0)
-  auto stage_chunk = [&](int64_t c) {
-    const int ws = (int)(c % kWordStages);
-    uint32_t *dw = W0 + ws * L.words_stage;
-    const int row = threadIdx.x >> 2, part = threadIdx.x & 3;
-    const int64_t m = m0 + row;
-    uint32_t *drow = dw + row * L.words_row;
-    if (m < a.M) {
-      const uint32_t *src = a.packed + m * a.wpr + c * L.words_row;
-      for (int k = part; k < B; k += 4) cp_async8(drow + 2 * k, src + 2 * k);
-    } else {
-      for (int k = part; k < B; k += 4) *reinterpret_cast<uint2 *>(drow + 2 * k) = make_uint2(0u, 0u);
-    }
-    if (threadIdx.x < kBK / 8)
-      cp_async16(S0 + ws * (kBK / 2) + 4 * threadIdx.x, a.sigma + c * (kBK / 2) + 4 * threadIdx.x);
-    cp_async_commit();
-  };
-
-  for (int i = threadIdx.x; i < a.N; i += kThreads) {
-    const float c0 = a.codebook[2 * i], c1 = a.codebook[2 * i + 1];
-    cbf[i] = make_float2(c0 + c1, c0 - c1);
+  for (int i = threadIdx.x; i < g.N; i += kThreads) {
+    const __half2 h = __floats2half2_rn(g.codebook[2 * i], g.codebook[2 * i + 1]);
+    cb[i] = *reinterpret_cast<const uint32_t *>(&h);
   }
-  if (threadIdx.x < 4 * kWordStages) {   // the padding words past the last row of each staging buffer
-    W0[(threadIdx.x >> 2) * L.words_stage + kBM * L.words_row + (threadIdx.x & 3)] = 0u;
-  }
-  // every column's factor d_j / (sqrt(b) s_j), once
-  for (int64_t j = threadIdx.x; j < a.K; j += kThreads) {
-    float f = __fdiv_rn(inv_sqrt_b, a.col_scale != nullptr ? a.col_scale[j] : 1.0f);
-    if (mask_is_negative(a.seed, j)) f = -f;
-    fac[j] = f;
-  }
+  if (threadIdx.x < 4 * SW)   // the words read past the last row of each stage
+    reinterpret_cast<uint32_t *>(W0 + (size_t)(threadIdx.x >> 2) * L.wpitch)[kBM * g.BW + (threadIdx.x & 3)] = 0u;
   if (threadIdx.x == 0) {
-    mbar_init(&bar_x[0], 1);
-    mbar_init(&bar_x[1], 1);
-    mbar_init(&bar_mma[0], 1);
-    mbar_init(&bar_mma[1], 1);
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&full_w[s], g.words_tma ? 1 : 32);
+      mbar_init(&empty_w[s], kDecWarps);
+    }
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&full_x[s], 1);
+      mbar_init(&full_a[s], kDecWarps);
+      mbar_init(&empty_a[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_fail = 0;
   }
@@ -230,226 +540,415 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gemm_kernel(const __grid_c
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (n_chunks > 0) stage_chunk(0);
-  if (n_chunks > 1) stage_chunk(1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  // instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N = NT, M = 128
-  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-
-  // this thread's item of every chunk: row rl = 8 w + lane / 4, columns 32 q .. 32 q + 31
-  const int q = lane & 3;
-  const int rl = 8 * warp + (lane >> 2);
-  const int64_t mrow = m0 + rl;
-  const bool rin = mrow < a.M;
-  const float rn = rin ? a.row_norm[mrow] : 0.0f;
-  uint32_t bad = (rin && !isfinite(rn)) ? QAMW_STATUS_NONFINITE_NORM : 0u;
-  const bool check_idx = a.N < (1 << B);
-  unsigned char *arow0 = A0 + (q >> 1) * kAtomBytesA + rl * 128;
-
+  uint32_t bad = 0;
   bool failed = false;
-  for (int64_t c = 0; c < n_chunks && !failed; ++c) {
-    const int s = (int)(c & 1);
-    unsigned char *Bs = B0 + s * L.stage_b;
-    if (c >= 2) {   // stage s was read by the MMAs of chunk c - 2 (every thread waits before overwriting it)
-      if (!mbar_wait(&bar_mma[s], (uint32_t)(((c - 2) >> 1) & 1), kWaitLimit)) bad |= QAMW_STATUS_TIMEOUT;
-    }
-    if (threadIdx.x == 0 && !(bad & QAMW_STATUS_TIMEOUT)) {
-      mbar_arrive_expect_tx(&bar_x[s], (uint32_t)L.stage_b);
-      tma_load_2d(Bs, &xmap, (int)(c * kBK), (int)t0, &bar_x[s]);
-      tma_load_2d(Bs + NT * 128, &xmap, (int)(c * kBK + 64), (int)t0, &bar_x[s]);
-    }
-    // the words of chunk c + 2 in flight while this one is decoded (its
-    // buffer held chunk c - 1, decoded before the previous barrier)
-    if (c + 2 < n_chunks) stage_chunk(c + 2);
-    if (c + 2 < n_chunks) cp_async_wait<2>();   // chunk c's words and sigma have landed
-    else if (c + 1 < n_chunks) cp_async_wait<1>();
-    else cp_async_wait<0>();
-    __syncthreads();
 
-    const int ws = (int)(c % kWordStages);
-    const uint32_t *rw = W0 + ws * L.words_stage + rl * L.words_row;
-    const float4 *sg4 = reinterpret_cast<const float4 *>(S0 + ws * (kBK / 2) + 16 * q);
-    uint32_t idx[16];
-    unpack16<BB>(rw, q, B, idx);
-    if (check_idx) {   // a codebook smaller than 2^B: out-of-range indices decode as centroid 0
+  if (warp < kDecWarps) {
+    // ---- decode: this thread's row rl and pairs 16 q .. 16 q + 15 of every chunk
+    const int q = lane & 3;
+    const int rl = 8 * warp + (lane >> 2);
+    const bool check_idx = g.N < (1 << B);
+    unsigned char *arow0 = A0 + (q >> 1) * kAtomBytes + rl * 128;
+    const bool hi = (q & 2) != 0;
+    int sa = 0, sw = 0;
+    uint32_t pa = 0, pw = 0;   // phase parities of the current stages
+    Cursor cur(u0, n_chunks, g.n_m);
+    for (int64_t u = u0; u < u1; ++u, cur.next(n_chunks, g.n_m)) {
+      const int c = cur.c;
+      const bool rin = cur.mt * kBM + rl < g.M;
+      // every failure decision is taken by the whole warp (the loop holds warp-wide syncs)
+      int r = wait_phase(&full_w[sw], pw, fail);
+      if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+      const int rem = g.words_tma ? ((c * 2 * B) & 3) : 0;
+      const uint32_t *rw = reinterpret_cast<const uint32_t *>(W0 + (size_t)sw * L.wpitch) + rl * g.BW + rem;
+      uint32_t idx[16];
+      unpack16<BB>(rw, q, B, idx);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_w[sw]);
+      uint32_t e[16];
 #pragma unroll
       for (int p = 0; p < 16; ++p) {
-        if (idx[p] >= (uint32_t)a.N) { bad |= QAMW_STATUS_BAD_INDEX; idx[p] = 0; }
+        uint32_t id = idx[p];
+        if (check_idx && id >= (uint32_t)g.N) {   // a codebook smaller than 2^B: decode as centroid 0
+          if (rin) bad |= QAMW_STATUS_BAD_INDEX;
+          id = 0;
+        }
+        e[p] = cb[id];
       }
+      if (u - u0 >= SA) {   // the stage's previous MMAs are done with it
+        r = wait_phase(&empty_a[sa], pa ^ 1u, fail);
+        if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+      }
+      // row rl, pairs 16 q .. + 15 = atom q / 2, 16-byte chunks 4 (q % 2) .. + 3;
+      // lanes with q >= 2 write their chunks in the order 2, 3, 0, 1, so that the
+      // 8 lanes of a quarter-warp (rows rl, rl + 1) hit 8 different bank groups
+      unsigned char *arow = arow0 + (size_t)sa * kStageBytesA;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const int ca = ch, cbk = ch ^ 2;
+        const uint4 va = make_uint4(e[4 * ca], e[4 * ca + 1], e[4 * ca + 2], e[4 * ca + 3]);
+        const uint4 vb = make_uint4(e[4 * cbk], e[4 * cbk + 1], e[4 * cbk + 2], e[4 * cbk + 3]);
+        const int cw = hi ? cbk : ca;
+        const int chunk16 = 4 * (q & 1) + cw;
+        *reinterpret_cast<uint4 *>(arow + ((chunk16 ^ (rl & 7)) << 4)) = hi ? vb : va;
+      }
+      fence_proxy_async_smem();   // the tile's generic stores become visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_a[sa]);
+      if (++sa == SA) { sa = 0; pa ^= 1u; }
+      if (++sw == SW) { sw = 0; pw ^= 1u; }
     }
-    float2 v[16];   // v[p] = r sigma_k (c0 + c1, c0 - c1): block bit 0 done, the row norm applied
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float4 sk = sg4[h];
-      const float sr[4] = {sk.x * rn, sk.y * rn, sk.z * rn, sk.w * rn};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[4 * h + u] = mul2(cbf[idx[4 * h + u]], make_float2(sr[u], sr[u]));
-    }
-    // block bits 1..4 in registers (pairs p and p | h/2), 5..6 across the 4 lanes of the row
-#pragma unroll
-    for (int t = 1; t < 5; ++t) {
-      if (t < log2b) {
-        const int h = 1 << (t - 1);
-#pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          if ((p & h) == 0) {
-            const float2 x0 = v[p], x1 = v[p | h];
-            v[p] = add2(x0, x1);
-            v[p | h] = sub2(x0, x1);
+  } else if (warp == kWarpWords) {
+    // ---- packed words of each unit -> word stage (u - u0) % SW
+    int sw = 0;
+    uint32_t pw = 0;
+    int64_t issued = 0;
+    Cursor cur(u0, n_chunks, g.n_m);
+    for (int64_t u = u0; u < u1; ++u, cur.next(n_chunks, g.n_m)) {
+      const int c = cur.c;
+      const int64_t m0 = cur.mt * kBM;
+      if (u - u0 >= SW) {
+        const int r = wait_phase(&empty_w[sw], pw ^ 1u, fail);
+        if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+      }
+      unsigned char *dst = W0 + (size_t)sw * L.wpitch;
+      if (g.words_tma) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full_w[sw], (uint32_t)(kBM * g.BW * 4));
+          tma_load_2d(dst, &wmap, (c * 2 * B) & ~3, (int)m0, &full_w[sw]);
+        }
+      } else {
+        // a row's 2B words of the chunk start 8-byte aligned (wpr and 2B are
+        // even); rows past M are not copied (their stale words decode to
+        // in-range centroids of rows that are never written)
+        for (int row = lane; row < kBM; row += 32) {
+          if (m0 + row < g.M) {
+            const uint32_t *src = g.packed + (m0 + row) * g.wpr + (int64_t)c * 2 * B;
+            uint32_t *d = reinterpret_cast<uint32_t *>(dst) + row * g.BW;
+            for (int k = 0; k < B; ++k) cp_async8(d + 2 * k, src + 2 * k);
           }
         }
+        cp_async_arrive_noinc(&full_w[sw]);
       }
+      issued = u - u0 + 1;
+      if (++sw == SW) { sw = 0; pw ^= 1u; }
     }
-#pragma unroll
-    for (int t = 5; t < 7; ++t) {
-      if (t < log2b) {
-        const int hb = 1 << (t - 5);
-        const float sgn = (lane & hb) ? -1.0f : 1.0f;
-        const float2 sg2 = make_float2(sgn, sgn);
-#pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[p].x, hb), __shfl_xor_sync(0xffffffffu, v[p].y, hb));
-          v[p] = fma2(sg2, v[p], o);
-        }
-      }
-    }
-    if (!rin) {
-#pragma unroll
-      for (int p = 0; p < 16; ++p) v[p] = make_float2(0.0f, 0.0f);
-    }
-    // scale by r d_j / (sqrt(b) s_j), round to bf16, store into the swizzled K-major tile:
-    // row rl, columns 32 q .. 32 q + 31 = atom q / 2, 16-byte chunks 4 (q % 2) .. + 3
-    unsigned char *arow = arow0 + s * kStageBytesA;
-    const float4 *f4 = reinterpret_cast<const float4 *>(fac + c * kBK + 32 * q);
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t pk[4];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float4 f = f4[2 * ch + h];
-        const float2 w0 = mul2(v[4 * ch + 2 * h], make_float2(f.x, f.y));
-        const float2 w1 = mul2(v[4 * ch + 2 * h + 1], make_float2(f.z, f.w));
-        const __nv_bfloat162 b0 = __floats2bfloat162_rn(w0.x, w0.y), b1 = __floats2bfloat162_rn(w1.x, w1.y);
-        pk[2 * h] = *reinterpret_cast<const uint32_t *>(&b0);
-        pk[2 * h + 1] = *reinterpret_cast<const uint32_t *>(&b1);
-      }
-      const int chunk16 = 4 * (q & 1) + ch;
-      *reinterpret_cast<uint4 *>(arow + ((chunk16 ^ (rl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-    fence_proxy_async_smem();   // the tile's generic stores become visible to the tensor cores
-    tc_fence_before();
-    if (__syncthreads_or(bad & QAMW_STATUS_TIMEOUT)) { failed = true; break; }
-    if (threadIdx.x == 0) {
-      if (!mbar_wait(&bar_x[s], (uint32_t)((c >> 1) & 1), kWaitLimit)) {
-        bad |= QAMW_STATUS_TIMEOUT;
-        s_fail = 1;
+    if (failed) {   // copies still in flight land before the CTA exits
+      if (g.words_tma) {
+        if (lane == 0)
+          for (int64_t i = (issued > SW ? issued - SW : 0); i < issued; ++i)
+            mbar_wait(&full_w[i % SW], (uint32_t)((i / SW) & 1), kWaitTries);
       } else {
+        cp_async_wait<0>();
+      }
+    }
+  } else if (warp == kWarpX) {
+    // ---- activation tile of each unit -> operand stage (u - u0) % SA
+    if (lane == 0) {
+      int sa = 0;
+      uint32_t pa = 0;
+      int64_t issued = 0;
+      griddep_wait();   // the a tiles are kernel 1's output
+      Cursor cur(u0, n_chunks, g.n_m);
+      for (int64_t u = u0; u < u1; ++u, cur.next(n_chunks, g.n_m)) {
+        const int c = cur.c;
+        const int64_t t0 = cur.tt * NT;
+        if (u - u0 >= SA) {
+          const int r = wait_phase(&empty_a[sa], pa ^ 1u, fail);
+          if (r) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+        }
+        unsigned char *dst = X0 + (size_t)sa * L.stage_x;
+        mbar_arrive_expect_tx(&full_x[sa], (uint32_t)L.stage_x);
+        tma_load_2d(dst, &xmap, c * kBK, (int)t0, &full_x[sa]);
+        tma_load_2d(dst + NT * 128, &xmap, c * kBK + 64, (int)t0, &full_x[sa]);
+        issued = u - u0 + 1;
+        if (++sa == SA) { sa = 0; pa ^= 1u; }
+      }
+      if (failed)
+        for (int64_t i = (issued > SA ? issued - SA : 0); i < issued; ++i)
+          mbar_wait(&full_x[i % SA], (uint32_t)((i / SA) & 1), kWaitTries);
+    }
+  } else if (warp == kWarpMma) {
+    // ---- MMA issue; segment = the CTA's units of one tile, accumulated in buffer seg % 2
+    if (lane == 0) {
+      // instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = NT, M = 128
+      const uint32_t idesc = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+      int sa = 0;
+      uint32_t pa = 0;
+      int64_t seg = 0;
+      bool any = false;
+      int c = (int)(u0 % n_chunks);
+      for (int64_t u = u0; u < u1; ++u, c = (c + 1 == n_chunks) ? 0 : c + 1) {
+        const bool first = (u == u0) || (c == 0);
+        const bool last = (u + 1 == u1) || (c == n_chunks - 1);
+        const uint32_t buf = (uint32_t)(seg & 1);
+        int r = 0;
+        if (first && seg >= 2) r = wait_phase(&acc_empty[buf], (uint32_t)(((seg >> 1) - 1) & 1), fail);
+        if (!r) r = wait_phase(&full_a[sa], pa, fail);
+        if (!r) r = wait_phase(&full_x[sa], pa, fail);
+        if (r) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(A0 + s * kStageBytesA), b_base = smem_u32(Bs);
+        const uint32_t a_base = smem_u32(A0 + (size_t)sa * kStageBytesA);
+        const uint32_t b_base = smem_u32(X0 + (size_t)sa * L.stage_x);
+        const uint32_t d = tmem + buf * acc_cols;
 #pragma unroll
         for (int k16 = 0; k16 < kBK / 16; ++k16) {
           const uint32_t atom = k16 >> 2, koff = (k16 & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(a_base + atom * kAtomBytesA + koff);
+          const uint64_t ad = smem_desc_sw128(a_base + atom * kAtomBytes + koff);
           const uint64_t bd = smem_desc_sw128(b_base + atom * (NT * 128) + koff);
-          mma_bf16(tmem, ad, bd, idesc, (c > 0 || k16 > 0) ? 1u : 0u);
+          mma_f16(d, ad, bd, idesc, (!first || k16 > 0) ? 1u : 0u);
         }
-        mma_commit(&bar_mma[s]);
+        mma_commit(&empty_a[sa]);
+        any = true;
+        if (last) {
+          mma_commit(&acc_full[buf]);
+          ++seg;
+        }
+        if (++sa == SA) { sa = 0; pa ^= 1u; }
       }
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-  if (s_fail) failed = true;
-  // the last chunk's commit covers every MMA before it
-  if (!failed && n_chunks > 0) {
-    const int64_t c = n_chunks - 1;
-    if (!mbar_wait(&bar_mma[c & 1], (uint32_t)((c >> 1) & 1), kWaitLimit)) {
-      bad |= QAMW_STATUS_TIMEOUT;
-      failed = true;
-    }
-  }
-  failed = __syncthreads_or(failed ? 1 : 0) != 0;
-  if (!failed) {
-    tc_fence_after();
-    // warps w, w + 4, w + 8, w + 12 read tensor-memory lanes 32 (w % 4) .. + 31 (rows), a quarter of the columns each
-    const int wq = warp & 3, grp = warp >> 2;
-    const int64_t m = m0 + 32 * wq + lane;
-    const int ncol = NT / 4;   // a multiple of 4
-    const int cbeg = grp * ncol, cend = cbeg + ncol;
-    // 16 columns per load; a load may reach 12 columns past the quarter (never
-    // past the allocated columns, which exceed NT by at least 16 unless the quarters are multiples of 16)
-    for (int c0 = cbeg; c0 < cend; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)c0, v);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int64_t t = t0 + c0 + j;
-        if (c0 + j < cend && m < a.M && t < g.T) g.Y[t * g.ldy + m] = v[j];
+      if (any) {   // every MMA issued completes before the tensor memory is freed
+        const int ls = (sa + SA - 1) % SA;                  // stage of the last committed unit
+        mbar_wait(&empty_a[ls], sa == 0 ? (pa ^ 1u) : pa, kWaitTries);
       }
     }
   } else {
-    // a wait ran out: give the copies and MMAs in flight a second bounded wait before freeing
-    if (threadIdx.x == 0) {
-      mbar_wait(&bar_x[0], 0, kWaitLimit);
-      mbar_wait(&bar_mma[0], 0, kWaitLimit);
+    // ---- epilogue warps: lanes 32 (warp % 4) .. + 31 of tensor memory = rows of the tile
+    const int wq = warp & 3;
+    const int row = 32 * wq + lane;
+    int64_t seg = 0;
+    int64_t u = u0;
+    griddep_wait();   // the token factors and the cleared counters are kernel 1's output
+    while (u < u1) {
+      const int64_t tile = u / n_chunks, c_begin = u - tile * n_chunks;
+      const int64_t seg_end = (u1 < (tile + 1) * n_chunks) ? u1 : (tile + 1) * n_chunks;
+      const bool whole = c_begin == 0 && seg_end == (tile + 1) * n_chunks;
+      const uint32_t buf = (uint32_t)(seg & 1);
+      // one decision for all 4 warps: the partial-sum path below holds their named barriers
+      const int r = wait_phase_sleep(&acc_full[buf], (uint32_t)((seg >> 1) & 1), fail);
+      if (epi_any(r != 0)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+      tc_fence_after();
+      const int64_t tt = tile / g.n_m;
+      const int64_t m = (tile - tt * g.n_m) * kBM + row;
+      const int64_t t0 = tt * NT;
+      const float rn = m < g.M ? g.row_norm[m] : 0.0f;
+      if (m < g.M && !isfinite(rn)) bad |= QAMW_STATUS_NONFINITE_NORM;
+      const uint32_t taddr = tmem + buf * acc_cols + ((uint32_t)(32 * wq) << 16);
+      if (whole) {
+        for (int c0 = 0; c0 < NT; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + (uint32_t)c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int64_t t = t0 + c0 + j;
+            if (m < g.M && t < g.T) g.Y[t * g.ldy + m] = (v[j] * rn) * g.tok_scale[t];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      } else {
+        // a part of the tile: this CTA's slot is 0 if the part is its first
+        // segment, else 1; the CTA that completes the tile adds all parts in
+        // the order of their CTAs
+        const int slot = (u == u0) ? 0 : 1;
+        float *mine = g.part + ((size_t)(2 * blockIdx.x + slot) * NT) * kBM;
+        for (int c0 = 0; c0 < NT; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + (uint32_t)c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) mine[(size_t)(c0 + j) * kBM + row] = v[j];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        const int64_t b_first = cta_of_unit(tile * n_chunks, G, g.n_units);
+        const int64_t b_last = cta_of_unit((tile + 1) * n_chunks - 1, G, g.n_units);
+        __threadfence();
+        epi_sync();
+        if (threadIdx.x == kWarpEpi * 32) {
+          const uint32_t old = atomicAdd(&g.counters[tile], 1u);
+          s_last = (old == (uint32_t)(b_last - b_first)) ? 1 : 0;
+          __threadfence();
+        }
+        epi_sync();
+        if (s_last) {
+          for (int c0 = 0; c0 < NT; c0 += 16) {
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            for (int64_t b = b_first; b <= b_last; ++b) {
+              // CTA b holds this tile in its first segment unless its range began in an earlier tile
+              const int sl = (range_start(b, G, g.n_units) < tile * n_chunks) ? 1 : 0;
+              const float *pp = g.part + ((size_t)(2 * b + sl) * NT) * kBM;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[j] += __ldcg(pp + (size_t)(c0 + j) * kBM + row);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int64_t t = t0 + c0 + j;
+              if (m < g.M && t < g.T) g.Y[t * g.ldy + m] = (acc[j] * rn) * g.tok_scale[t];
+            }
+          }
+        }
+        epi_sync();   // s_last is read by all before the next part overwrites it
+      }
+      ++seg;
+      u = seg_end;
     }
   }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols)
                               : "memory");
   bad = __reduce_or_sync(0xffffffffu, bad);
-  if (lane == 0) status_or(a.status, bad);
+  if (lane == 0) status_or(g.status, bad);
 }
 
 }  // namespace
 
-size_t decode_gemm_smem_bytes(int NT, int N, int B, int64_t K) { return 1024 + gemm_smem(NT, N, B, K).total; }
+size_t decode_matmul_workspace_bytes(int64_t M, int64_t K, int64_t T) { return ws_layout(M, K, T).total; }
 
 cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
-                               cudaStream_t s) {
+                               void *workspace, cudaStream_t s) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
   int dev = 0, smem_max = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-  // the widest token tile (<= 256, a multiple of 16) whose stages fit
-  int NT = (int)std::min<int64_t>(256, (T + 15) / 16 * 16);
-  while (NT > 16 && decode_gemm_smem_bytes(NT, d.N, d.bits, d.K) + 256 > (size_t)smem_max) NT -= 16;
-  if (decode_gemm_smem_bytes(NT, d.N, d.bits, d.K) + 256 > (size_t)smem_max) return cudaErrorNotSupported;
-  CUtensorMap xmap;
+  const WsLayout W = ws_layout(d.M, d.K, T);
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  __half *A = reinterpret_cast<__half *>(ws);
+  float *tok_scale = reinterpret_cast<float *>(ws + W.off_scale);
+  uint32_t *counters = reinterpret_cast<uint32_t *>(ws + W.off_cnt);
+  float *part = reinterpret_cast<float *>(ws + W.off_part);
+
+  // ---- kernel 2 shapes (kernel 1 clears its tile counters)
+  GemmArgs g;
+  g.packed = d.packed;
+  g.row_norm = d.row_norm;
+  g.codebook = d.codebook;
+  g.tok_scale = tok_scale;
+  g.counters = counters;
+  g.part = part;
+  g.Y = Y;
+  g.ldy = ldy;
+  g.M = d.M;
+  g.K = d.K;
+  g.T = T;
+  g.wpr = d.wpr;
+  g.N = d.N;
+  g.bits = d.bits;
+  g.status = d.status;
+  const int B = d.bits;
+  // the packed words by TMA when the row pitch is a multiple of 16 bytes: a
+  // chunk's 2B words start at word 2Bc, i.e. 0 or 2 words past a 16-byte
+  // boundary, so a box of 2B + 2 words (rounded up to 4) holds them
+  g.words_tma = ((d.wpr * 4) % 16 == 0 && reinterpret_cast<uintptr_t>(d.packed) % 16 == 0) ? 1 : 0;
+  g.BW = g.words_tma ? ((2 * B + 2 + 3) & ~3) : 2 * B;
+  // the widest token tile (<= 256, a multiple of 16) whose stages fit; 2 to
+  // 4 operand stages and 3 to 6 word stages
+  const int64_t budget = (int64_t)smem_max - 1024 - 256 - kPrepSmemReserve;
+  int NT = nt_cap(T);
+  int SA = 4, SW = 6;
+  auto fits = [&](int nt, int sa, int sw) { return (int64_t)gemm_smem(nt, sa, sw, g.BW, d.N).total <= budget; };
+  while (!fits(NT, SA, SW)) {
+    if (SW > 3) --SW;
+    else if (SA > 2) --SA;
+    else if (NT > 16) NT -= 16;
+    else return cudaErrorNotSupported;
+  }
+  g.NT = NT;
+  g.SA = SA;
+  g.SW = SW;
+  g.n_m = (d.M + kBM - 1) / kBM;
+  const int64_t n_tiles = g.n_m * ((T + NT - 1) / NT);
+  g.n_units = n_tiles * (d.K / kBK);
+  const int64_t G = std::min<int64_t>(std::min<int64_t>(sm_count(), kMaxCtas), g.n_units);
+
+  // ---- kernel 1: a cluster of S CTAs per token
+  {
+    PrepArgs p;
+    p.X = X;
+    p.ldx = ldx;
+    p.T = T;
+    p.K = d.K;
+    p.sigma = d.sigma;
+    p.col_scale = d.col_scale;
+    p.seed = d.seed;
+    p.log2b = d.log2b;
+    p.A = A;
+    p.tok_scale = tok_scale;
+    p.counters = counters;
+    p.n_counters = n_tiles;
+    const int ucols = d.log2b > 9 ? (1 << d.log2b) : 512;
+    const int64_t n_units = (d.K + ucols - 1) / ucols;
+    p.S = (int)std::min<int64_t>(kPrepCluster, n_units);
+    const size_t smem = (size_t)((n_units + p.S - 1) / p.S) * ucols * 4;
+    if ((e = set_max_dynamic_smem(reinterpret_cast<const void *>(prepare_x_kernel), smem)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.S * T), 1, 1);
+    cfg.blockDim = dim3(kPrepThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, prepare_x_kernel, p)) != cudaSuccess) return e;
+  }
+
+  CUtensorMap xmap, wmap;
   {
     cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)T};
-    cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)d.K * 2};
     cuuint32_t box[2] = {64, (cuuint32_t)NT};
     cuuint32_t es[2] = {1, 1};
-    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(X), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  GemmArgs g;
-  g.d = d;
-  g.T = T;
-  g.NT = NT;
-  g.Y = Y;
-  g.ldy = ldy;
-  const size_t smem = decode_gemm_smem_bytes(NT, d.N, d.bits, d.K);
-  const dim3 grid((unsigned)((d.M + kBM - 1) / kBM), (unsigned)((T + NT - 1) / NT));
-  // 11- and 10-bit codes with 128-column blocks compiled for their shape; anything else at run time
+  if (g.words_tma) {
+    cuuint64_t dims[2] = {(cuuint64_t)d.wpr, (cuuint64_t)d.M};
+    cuuint64_t strides[1] = {(cuuint64_t)d.wpr * 4};
+    cuuint32_t box[2] = {(cuuint32_t)g.BW, (cuuint32_t)kBM};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(d.packed), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    wmap = xmap;   // unused
+  }
+  const size_t smem = 1024 + gemm_smem(NT, SA, SW, g.BW, d.N).total;
   auto run = [&](auto kern) -> cudaError_t {
     cudaError_t err = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, smem, s>>>(xmap, g);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)G, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, xmap, wmap, g);
   };
-  if (d.bits == 11 && d.log2b == 7) return run(decode_gemm_kernel<11, 7>);
-  if (d.bits == 10 && d.log2b == 7) return run(decode_gemm_kernel<10, 7>);
-  return run(decode_gemm_kernel<0, 0>);
+  // 11- and 10-bit codes compiled for their shape; anything else at run time
+  if (B == 11) return run(decode_gemm_kernel<11>);
+  if (B == 10) return run(decode_gemm_kernel<10>);
+  return run(decode_gemm_kernel<0>);
 }
 
 }  // namespace qamw

@@ -164,12 +164,13 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 bool decode_tma_applicable(const DecodeArgs &a);
 cudaError_t launch_decode_tma(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_rotate_test(const RotateTestArgs &a, cudaStream_t s);
-// Decode fused with Y = X W_bf16^T on the tensor cores (qamw_decode_gemm.cu):
-// X bf16 [T][ldx], Y fp32 [T][ldy]; K % 128 == 0, b <= 128, N <= 2048; cudaErrorNotSupported
-// if K is too wide for the shared-memory factor table.
-size_t decode_gemm_smem_bytes(int NT, int N, int B, int64_t K);
+// Decode fused with the matrix multiply Y = X W_hat^T on the tensor cores
+// (qamw_decode_gemm.cu): X bf16 [T][ldx], Y fp32 [T][ldy], workspace of
+// decode_matmul_workspace_bytes(M, K, T) bytes (256-byte aligned); K % 128 == 0,
+// K <= 32768, N <= QAMW_MAX_CENTROIDS, T <= 2^24.
+size_t decode_matmul_workspace_bytes(int64_t M, int64_t K, int64_t T);
 cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T, int64_t ldx, float *Y, int64_t ldy,
-                               cudaStream_t s);
+                               void *workspace, cudaStream_t s);
 // The same for b <= 512 with the 512-column rotation of the encode and calibrate kernels.
 cudaError_t launch_rotate_test512(const RotateTestArgs &a, cudaStream_t s);
 
