@@ -2,12 +2,13 @@
 // QAM-W Codec", QAM-W Technical Summary) for Hadamard blocks b <= 512.
 //
 // sigma_k = RN32(sqrt(2/pi) * (1/M) * sum_i ||z_ik||) over the rotated unit
-// rows. A CTA of 28 warps takes a contiguous range of tiles (28 rows x one
-// 512-column chunk) in chunk-major order, warp w holding row 28g + w with the
-// 512-column unit of qamw_rotate16.cuh (half-size transpose buffers, so that
-// 28 warps fit beside the staging of |z|). The 28 rows' ||z_ik|| are added in
-// shared memory in row order (w = 0..27) and written as the row group's fp64
-// partial sum; sigma_reduce (qamw_encode.cu) adds the groups in a fixed order.
+// rows. A CTA of 14 warps takes a contiguous range of tiles (28 rows x one
+// 512-column chunk) in chunk-major order; warp w rotates rows 28g + w and
+// 28g + w + 14 with the 512-column unit of qamw_rotate16.cuh (one-pass
+// transposes; the block size fixed at compile time for bf16 weights). The 28
+// rows' ||z_ik|| are added in shared memory in row order (0..27) and written
+// as the row group's fp64 partial sum; sigma_reduce (qamw_encode.cu) adds the
+// groups in a fixed order.
 // The sums are the same, in the same order, as those of the 1024-column
 // calibrate kernel (b = 1024), so sigma does not depend on the kernel.
 #include <algorithm>

@@ -60,7 +60,7 @@ namespace {
 
 constexpr int kBM = 128;                   // output rows per tile (tensor-memory lanes)
 constexpr int kBK = 128;                   // columns (64 pairs) per chunk
-constexpr int kDecWarps = 16;              // thread: row 8 w + lane / 4, pairs 16 (lane % 4) .. + 15
+constexpr int kDecWarps = 16;              // SA groups (4 or 2); a group decodes one unit at a time
 constexpr int kWarpWords = kDecWarps;      // streams the packed words
 constexpr int kWarpX = kDecWarps + 1;      // streams the activation tiles
 constexpr int kWarpMma = kDecWarps + 2;    // issues the MMAs
@@ -73,7 +73,6 @@ constexpr int kMaxCtas = 160;              // persistent CTAs at most (the parti
 constexpr uint32_t kWaitTries = 1u << 22;  // try_wait attempts before a spinning wait gives up
 constexpr uint32_t kSleepTries = 1u << 21; // attempts (<= 512 ns apart) before a sleeping wait gives up
 constexpr int kPrepThreads = 128;          // small enough to share an SM with a CTA of kernel 2
-constexpr int kPrepSmemReserve = 18 * 1024;   // shared memory kernel 2 leaves to one CTA of kernel 1
 constexpr int kPrepCluster = 8;            // CTAs per token in kernel 1 (portable cluster size)
 
 // ---------------------------------------------------------------------------
@@ -107,8 +106,8 @@ struct GemmArgs {
   int64_t n_units;          // tiles x chunks
   int N, bits;
   int NT;                   // tokens per tile (16..256, a multiple of 16)
-  int SA;                   // operand stages (weight tile + activation tile)
-  int SW;                   // word stages
+  int SA;                   // operand stages (weight tile + activation tile) = decode groups (4 or 2)
+  int SW;                   // word stages (a multiple of SA)
   int BW;                   // staged words per row and chunk
   int words_tma;            // 1: words by TMA; 0: by cp.async
   int32_t *status;
@@ -252,39 +251,70 @@ struct Cursor {
   }
 };
 
-// The 16 indices of pairs 16 q .. 16 q + 15 of a row's chunk, from its 2B
-// staged words (LSB-first B-bit fields). BB > 0: B fixed at compile time (the
-// quarter's first field starts at bit 0 or 16 of a word; a 16-bit funnel
-// shift aligns it, and every later position is a constant).
+// The operand row of one unit: the 64 fp16 centroid pairs of row rl, written
+// in the 128-byte swizzled K-major layout (pairs 16 j .. 16 j + 15 = atom
+// j / 2, 16-byte chunks 4 (j % 2) .. + 3; chunk position XOR rl % 8, so the 8
+// rows of a quarter-warp hit 8 different bank groups). Field k of the row's
+// chunk is bits 32 REM + k BB .. of the staged words w. Returns the status bits.
 template <int BB>
-__device__ __forceinline__ void unpack16(const uint32_t *rw, int q, int B, uint32_t (&idx)[16]) {
-  if (BB > 0) {
-    constexpr int kNW = (16 * BB + 31) / 32 + 1;
-    const int bit0 = 16 * q * BB;
-    const uint32_t *p = rw + (bit0 >> 5);
-    uint32_t w[kNW + 1];
+struct RowWords {
+  static constexpr int kNW4 = (64 + 64 * BB + 127) / 128;   // 16-byte loads that cover REM <= 2 plus 64 fields
+};
+template <int BB, int REM>
+__device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<BB>::kNW4], const uint32_t *cb,
+                                              unsigned char *arow, int rl, int jb, int nb, bool check_idx, int N,
+                                              bool rin) {
+  uint32_t bad = 0;
 #pragma unroll
-    for (int i = 0; i <= kNW; ++i) w[i] = p[i];
-    if (bit0 & 31) {
+  for (int j = 0; j < 4; ++j) {
+    if (j < jb || j >= jb + nb) continue;   // the batches of this thread's part of the row
+    uint32_t e[16];
 #pragma unroll
-      for (int i = 0; i < kNW; ++i) w[i] = __funnelshift_r(w[i], w[i + 1], 16);
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int b = k * BB, wi = b >> 5, sh = b & 31;
+    for (int p = 0; p < 16; ++p) {
+      const int b = 32 * REM + (16 * j + p) * BB, wi = b >> 5, sh = b & 31;
       uint32_t v = w[wi] >> sh;
       if (sh + BB > 32) v |= w[wi + 1] << (32 - sh);
-      idx[k] = v & ((1u << BB) - 1u);
+      uint32_t id = v & ((1u << BB) - 1u);
+      if (check_idx && id >= (uint32_t)N) {   // a codebook smaller than 2^B: decode as centroid 0
+        if (rin) bad |= QAMW_STATUS_BAD_INDEX;
+        id = 0;
+      }
+      e[p] = cb[id];
     }
-  } else {
+    unsigned char *atom = arow + (j >> 1) * kAtomBytes;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int b = (16 * q + k) * B, wi = b >> 5, sh = b & 31;
-      uint64_t v = rw[wi];
-      if (sh + B > 32) v |= (uint64_t)rw[wi + 1] << 32;
-      idx[k] = (uint32_t)(v >> sh) & ((1u << B) - 1u);
-    }
+    for (int ch = 0; ch < 4; ++ch)
+      *reinterpret_cast<uint4 *>(atom + (((4 * (j & 1) + ch) ^ (rl & 7)) << 4)) =
+          make_uint4(e[4 * ch], e[4 * ch + 1], e[4 * ch + 2], e[4 * ch + 3]);
   }
+  return bad;
+}
+// the same for a code size known only at run time (fields read from shared memory)
+__device__ __forceinline__ uint32_t write_row_any(const uint32_t *rowp, int rem, int B, const uint32_t *cb,
+                                                  unsigned char *arow, int rl, int jb, int nb, bool check_idx,
+                                                  int N, bool rin) {
+  uint32_t bad = 0;
+  for (int j = jb; j < jb + nb; ++j) {
+    uint32_t e[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const int b = 32 * rem + (16 * j + p) * B, wi = b >> 5, sh = b & 31;
+      uint64_t v = rowp[wi];
+      if (sh + B > 32) v |= (uint64_t)rowp[wi + 1] << 32;
+      uint32_t id = (uint32_t)(v >> sh) & ((1u << B) - 1u);
+      if (check_idx && id >= (uint32_t)N) {
+        if (rin) bad |= QAMW_STATUS_BAD_INDEX;
+        id = 0;
+      }
+      e[p] = cb[id];
+    }
+    unsigned char *atom = arow + (j >> 1) * kAtomBytes;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch)
+      *reinterpret_cast<uint4 *>(atom + (((4 * (j & 1) + ch) ^ (rl & 7)) << 4)) =
+          make_uint4(e[4 * ch], e[4 * ch + 1], e[4 * ch + 2], e[4 * ch + 3]);
+  }
+  return bad;
 }
 
 // ----------------------------------------------------------------------------
@@ -520,11 +550,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW; ++s) {
       mbar_init(&full_w[s], g.words_tma ? 1 : 32);
-      mbar_init(&empty_w[s], kDecWarps);
+      mbar_init(&empty_w[s], kDecWarps / SA);   // the warps of the group that decodes the stage's units
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(&full_x[s], 1);
-      mbar_init(&full_a[s], kDecWarps);
+      mbar_init(&full_a[s], kDecWarps / SA);
       mbar_init(&empty_a[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -548,59 +578,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool failed = false;
 
   if (warp < kDecWarps) {
-    // ---- decode: this thread's row rl and pairs 16 q .. 16 q + 15 of every chunk
-    const int q = lane & 3;
-    const int rl = 8 * warp + (lane >> 2);
+    // ---- decode: SA groups of 16 / SA warps; group grp takes the CTA's units
+    // u0 + grp, u0 + grp + SA, ... into operand stage grp and word stages
+    // grp, grp + SA, ... (each stage is used by one group, in order), so SA
+    // units are decoded at once. In a unit, thread tg of the group owns row
+    // rl = tg % 128 and batches jb .. jb + nb - 1 of its 4 batches of 16 pairs.
+    const int wpg = kDecWarps / SA;
+    const int grp = warp / wpg;
+    const int tg = (warp % wpg) * 32 + lane;
+    const int rl = tg & (kBM - 1);
+    const int nb = SA;                 // batches per thread: 4 (SA = 4, one thread per row) or 2 (two)
+    const int jb = (tg >> 7) * nb;
     const bool check_idx = g.N < (1 << B);
-    unsigned char *arow0 = A0 + (q >> 1) * kAtomBytes + rl * 128;
-    const bool hi = (q & 2) != 0;
-    int sa = 0, sw = 0;
-    uint32_t pa = 0, pw = 0;   // phase parities of the current stages
-    Cursor cur(u0, n_chunks, g.n_m);
-    for (int64_t u = u0; u < u1; ++u, cur.next(n_chunks, g.n_m)) {
+    int sw = grp;
+    uint32_t qa = 0, qw = 0;   // stage use counts (phase = count & 1)
+    unsigned char *arow = A0 + (size_t)grp * kStageBytesA + rl * 128;
+    Cursor cur(u0 + grp, n_chunks, g.n_m);
+    for (int64_t u = u0 + grp; u < u1; u += SA) {
       const int c = cur.c;
       const bool rin = cur.mt * kBM + rl < g.M;
       // every failure decision is taken by the whole warp (the loop holds warp-wide syncs)
-      int r = wait_phase(&full_w[sw], pw, fail);
+      int r = wait_phase(&full_w[sw], qw & 1u, fail);
       if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
-      const int rem = g.words_tma ? ((c * 2 * B) & 3) : 0;
-      const uint32_t *rw = reinterpret_cast<const uint32_t *>(W0 + (size_t)sw * L.wpitch) + rl * g.BW + rem;
-      uint32_t idx[16];
-      unpack16<BB>(rw, q, B, idx);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_w[sw]);
-      uint32_t e[16];
+      const int rem = g.words_tma ? ((c * 2 * B) & 3) : 0;   // the chunk's first word in the staged row
+      const uint32_t *rowp = reinterpret_cast<const uint32_t *>(W0 + (size_t)sw * L.wpitch) + rl * g.BW;
+      if (BB > 0) {
+        constexpr int kNW4 = RowWords<BB>::kNW4;
+        uint32_t w[4 * kNW4];
+        const uint4 *src = reinterpret_cast<const uint4 *>(rowp);   // 16-byte rows, BW / 4 odd: no bank conflict
 #pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        uint32_t id = idx[p];
-        if (check_idx && id >= (uint32_t)g.N) {   // a codebook smaller than 2^B: decode as centroid 0
-          if (rin) bad |= QAMW_STATUS_BAD_INDEX;
-          id = 0;
+        for (int i = 0; i < kNW4; ++i) {
+          const uint4 v = src[i];
+          w[4 * i] = v.x;
+          w[4 * i + 1] = v.y;
+          w[4 * i + 2] = v.z;
+          w[4 * i + 3] = v.w;
         }
-        e[p] = cb[id];
-      }
-      if (u - u0 >= SA) {   // the stage's previous MMAs are done with it
-        r = wait_phase(&empty_a[sa], pa ^ 1u, fail);
-        if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
-      }
-      // row rl, pairs 16 q .. + 15 = atom q / 2, 16-byte chunks 4 (q % 2) .. + 3;
-      // lanes with q >= 2 write their chunks in the order 2, 3, 0, 1, so that the
-      // 8 lanes of a quarter-warp (rows rl, rl + 1) hit 8 different bank groups
-      unsigned char *arow = arow0 + (size_t)sa * kStageBytesA;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int ca = ch, cbk = ch ^ 2;
-        const uint4 va = make_uint4(e[4 * ca], e[4 * ca + 1], e[4 * ca + 2], e[4 * ca + 3]);
-        const uint4 vb = make_uint4(e[4 * cbk], e[4 * cbk + 1], e[4 * cbk + 2], e[4 * cbk + 3]);
-        const int cw = hi ? cbk : ca;
-        const int chunk16 = 4 * (q & 1) + cw;
-        *reinterpret_cast<uint4 *>(arow + ((chunk16 ^ (rl & 7)) << 4)) = hi ? vb : va;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_w[sw]);
+        if (qa > 0) {   // the stage's previous MMAs are done with it
+          r = wait_phase(&empty_a[grp], (qa & 1u) ^ 1u, fail);
+          if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+        }
+        if (rem == 0) bad |= write_row<BB, 0>(w, cb, arow, rl, jb, nb, check_idx, g.N, rin);
+        else bad |= write_row<BB, 2>(w, cb, arow, rl, jb, nb, check_idx, g.N, rin);
+      } else {
+        if (qa > 0) {
+          r = wait_phase(&empty_a[grp], (qa & 1u) ^ 1u, fail);
+          if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+        }
+        bad |= write_row_any(rowp, rem, B, cb, arow, rl, jb, nb, check_idx, g.N, rin);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_w[sw]);
       }
       fence_proxy_async_smem();   // the tile's generic stores become visible to the tensor cores
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full_a[sa]);
-      if (++sa == SA) { sa = 0; pa ^= 1u; }
-      if (++sw == SW) { sw = 0; pw ^= 1u; }
+      if (lane == 0) mbar_arrive(&full_a[grp]);
+      for (int k = 0; k < SA; ++k) cur.next(n_chunks, g.n_m);
+      ++qa;
+      sw += SA;
+      if (sw >= SW) { sw -= SW; ++qw; }
     }
   } else if (warp == kWarpWords) {
     // ---- packed words of each unit -> word stage (u - u0) % SW
@@ -848,20 +885,31 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   const int B = d.bits;
   // the packed words by TMA when the row pitch is a multiple of 16 bytes: a
   // chunk's 2B words start at word 2Bc, i.e. 0 or 2 words past a 16-byte
-  // boundary, so a box of 2B + 2 words (rounded up to 4) holds them
+  // boundary, so a box of 2B + 2 words (rounded up to 4) holds them; cp.async
+  // copies place them at the start of the staged row
   g.words_tma = ((d.wpr * 4) % 16 == 0 && reinterpret_cast<uintptr_t>(d.packed) % 16 == 0) ? 1 : 0;
-  g.BW = g.words_tma ? ((2 * B + 2 + 3) & ~3) : 2 * B;
-  // the widest token tile (<= 256, a multiple of 16) whose stages fit; 2 to
-  // 4 operand stages and 3 to 6 word stages
-  const int64_t budget = (int64_t)smem_max - 1024 - 256 - kPrepSmemReserve;
-  int NT = nt_cap(T);
-  int SA = 4, SW = 6;
+  g.BW = (2 * B + 2 + 3) & ~3;
+  if ((g.BW / 4) % 2 == 0) g.BW += 4;   // an odd number of 16-byte groups per row: rows hit different banks
+  // kernel 1's CTA shape, and the shared memory kernel 2 leaves to one of its
+  // CTAs (so that it can run beside kernel 2)
+  const int ucols = d.log2b > 9 ? (1 << d.log2b) : 512;
+  const int64_t prep_units = (d.K + ucols - 1) / ucols;
+  const int prep_S = (int)std::min<int64_t>(kPrepCluster, prep_units);
+  const size_t prep_smem = (size_t)((prep_units + prep_S - 1) / prep_S) * ucols * 4;
+  const int64_t budget = (int64_t)smem_max - 1024 - 256 - (int64_t)prep_smem - 2048;
+  // up to 16 tokens: 4 decode groups (4 units in flight) and 16-token tiles;
+  // more tokens: 2 groups and the widest token tile (<= 256, a multiple of
+  // 16) whose stages fit; word stages 1 or 2 per group
   auto fits = [&](int nt, int sa, int sw) { return (int64_t)gemm_smem(nt, sa, sw, g.BW, d.N).total <= budget; };
-  while (!fits(NT, SA, SW)) {
-    if (SW > 3) --SW;
-    else if (SA > 2) --SA;
-    else if (NT > 16) NT -= 16;
-    else return cudaErrorNotSupported;
+  int NT = nt_cap(T), SA = 4, SW = 4;
+  if (!(NT == 16 && fits(NT, 4, 4))) {
+    SA = 2;
+    SW = 4;
+    while (!fits(NT, SA, SW)) {
+      if (SW > 2) SW = 2;
+      else if (NT > 16) NT -= 16;
+      else return cudaErrorNotSupported;
+    }
   }
   g.NT = NT;
   g.SA = SA;
@@ -886,10 +934,8 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
     p.tok_scale = tok_scale;
     p.counters = counters;
     p.n_counters = n_tiles;
-    const int ucols = d.log2b > 9 ? (1 << d.log2b) : 512;
-    const int64_t n_units = (d.K + ucols - 1) / ucols;
-    p.S = (int)std::min<int64_t>(kPrepCluster, n_units);
-    const size_t smem = (size_t)((n_units + p.S - 1) / p.S) * ucols * 4;
+    p.S = prep_S;
+    const size_t smem = prep_smem;
     if ((e = set_max_dynamic_smem(reinterpret_cast<const void *>(prepare_x_kernel), smem)) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.S * T), 1, 1);
