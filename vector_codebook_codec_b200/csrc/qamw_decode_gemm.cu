@@ -13,11 +13,11 @@
 //   a_t[i]  = sigma_{i/2} (H_b (d (.) X[t] / s))_i / sqrt(b)      (per block of b columns),
 // which costs log2 b adds per activation instead of per weight.
 //
-// Kernel 1 (prepare_x_kernel): a cluster of up to 8 CTAs per token computes
-// a_t in fp32 (each CTA a share of the columns), agrees on the token's
-// largest |a| through distributed shared memory, scales by 2^-e_t so that it
-// lies in (2^13, 2^14], and stores fp16 a_t and 2^e_t. It also clears the
-// tile counters of kernel 2.
+// Kernel 1 (prepare_x_kernel): a cluster of up to 8 CTAs per token (one CTA
+// from 512 tokens on) computes a_t in fp32 (each CTA a share of the columns),
+// agrees on the token's largest |a| through distributed shared memory,
+// scales by 2^-e_t so that it lies in (2^13, 2^14], and stores fp16 a_t and
+// 2^e_t. It also clears the tile counters of kernel 2.
 //
 // Kernel 2 (decode_gemm_kernel), persistent: one CTA per SM. The work is the
 // list of (output tile, K chunk) units -- an output tile is 128 rows m x NT
@@ -383,6 +383,12 @@ __global__ void __launch_bounds__(kPrepThreads, 10) prepare_x_kernel(PrepArgs p)
     const int64_t col = (rank + li * S) * (int64_t)ucols + part * 512 + 16 * lane;
     float *dst = vloc + li * ucols + part * 512 + 16 * lane;
     const bool in = col < K;   // K % 16 == 0: a lane's 16 columns are all in or all out
+    float4 sg4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    if (lb <= 9 && in) {   // sigma of the lane's 8 pairs, loaded early (col % 16 == 0: 32-byte aligned)
+      const float4 *sg = reinterpret_cast<const float4 *>(p.sigma + (col >> 1));
+      sg4[0] = sg[0];
+      sg4[1] = sg[1];
+    }
     float u[16];
     if (in) {
       const uint4 *src = reinterpret_cast<const uint4 *>(xr + col);
@@ -420,10 +426,9 @@ __global__ void __launch_bounds__(kPrepThreads, 10) prepare_x_kernel(PrepArgs p)
       for (int e = 0; e < 16; ++e) u[e] = __fmaf_rn(sgn, u[e], __shfl_xor_sync(0xffffffffu, u[e], h));
     }
     if (lb <= 9 && in) {   // every butterfly done: times sigma_k / sqrt(b) here
-      const float4 *sg = reinterpret_cast<const float4 *>(p.sigma + (col >> 1));   // col % 16 == 0: 32-byte aligned
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const float4 s4 = sg[h];
+        const float4 s4 = sg4[h];
         const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -895,13 +900,16 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   g.words_tma = ((d.wpr * 4) % 16 == 0 && reinterpret_cast<uintptr_t>(d.packed) % 16 == 0) ? 1 : 0;
   g.BW = (B + 3 + 3) & ~3;
   if ((g.BW / 4) % 2 == 0) g.BW += 4;   // an odd number of 16-byte groups per row: rows hit different banks
-  // kernel 1's CTA shape, and the shared memory kernel 2 leaves to one of its
-  // CTAs (so that it can run beside kernel 2)
+  // kernel 1's CTA shape: a cluster of up to 8 CTAs per token for few tokens
+  // (its latency is on the critical path), one CTA per token from 512 tokens
+  // on (enough CTAs to fill the GPU without clusters); for few tokens kernel
+  // 2 leaves shared memory to one CTA of kernel 1, so that it can start
+  // beside it
   const int ucols = d.log2b > 9 ? (1 << d.log2b) : 512;
   const int64_t prep_units = (d.K + ucols - 1) / ucols;
-  const int prep_S = (int)std::min<int64_t>(kPrepCluster, prep_units);
+  const int prep_S = T >= 512 ? 1 : (int)std::min<int64_t>(kPrepCluster, prep_units);
   const size_t prep_smem = (size_t)((prep_units + prep_S - 1) / prep_S) * ucols * 4;
-  const int64_t budget = (int64_t)smem_max - 1024 - 256 - (int64_t)prep_smem - 2048;
+  const int64_t budget = (int64_t)smem_max - 1024 - 256 - (prep_S > 1 ? (int64_t)prep_smem + 2048 : 0);
   // the widest token tile (<= 256, a multiple of 16) and, for it, the first
   // stage counts of this list that fit: 4 decode groups before 2, word
   // stages 2 then 1 per group, activation stages 8 .. 2
