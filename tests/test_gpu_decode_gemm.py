@@ -121,6 +121,34 @@ def test_fused_decode_matmul_matches_the_oracle(M, K, T, block, N, bits):
     _check(M, K, T, block, N, bits, seed=M + K + T)
 
 
+def test_fused_decode_matmul_many_tokens():
+    """600 tokens: the activation kernel runs one CTA per token (from 512 on)
+    and the output has three 256-token tiles, the last one ragged."""
+    _check(256, 512, 600, 128, 2048, 11, seed=21)
+
+
+def test_fused_decode_matmul_single_row_and_strided_operands():
+    """M = 1 (one row tile, 127 rows past M) and activations / outputs with
+    leading dimensions larger than K / M."""
+    M, K, T = 1, 256, 5
+    enc, Cd, Xb, idx, r, sig, s, C = _case(M, K, T, 128, 2048, 11, seed=31)
+    Xpad = torch.zeros((T, K + 64), dtype=torch.bfloat16)
+    Xpad[:, :K] = Xb
+    Xs = Xpad.cuda()[:, :K]                       # ldx = K + 64
+    Ypad = torch.full((T, M + 7), -7.0, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qamw.decode_matmul(enc, Cd, Xs, status=st, out=Ypad[:, :M])
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.all(Ypad[:, M:] == -7.0)          # nothing written past M
+    Y = Ypad[:, :M].cpu().numpy().astype(np.float64)
+    Wh = codec.decode_with_scale(idx, r, sig, s, K, 128, 31, C)
+    X64 = Xb.to(torch.float64).numpy()
+    ref = X64 @ Wh.T
+    bound = _bound(X64, idx, r, sig, s, C, K, 128, 31, np.arange(M)) + 2.0 ** -22 * np.abs(ref) + 1e-30
+    assert np.all(np.abs(Y - ref) <= bound)
+
+
 def test_fused_decode_matmul_without_channel_scale():
     _check(256, 512, 16, 128, 2048, 11, seed=3, with_scale=False)
 

@@ -106,7 +106,7 @@ struct GemmArgs {
   int64_t n_units;          // tiles x chunks
   int N, bits;
   int NT;                   // tokens per tile (16..256, a multiple of 16)
-  int SA;                   // weight-tile stages = decode groups (4 or 2)
+  int SA;                   // weight-tile stages = decode groups (4)
   int SW;                   // word stages (a multiple of SA)
   int SX;                   // activation-tile stages
   int BW;                   // staged words per row and chunk
@@ -911,13 +911,13 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   const size_t prep_smem = (size_t)((prep_units + prep_S - 1) / prep_S) * ucols * 4;
   const int64_t budget = (int64_t)smem_max - 1024 - 256 - (prep_S > 1 ? (int64_t)prep_smem + 2048 : 0);
   // the widest token tile (<= 256, a multiple of 16) and, for it, the first
-  // stage counts of this list that fit: 4 decode groups before 2, word
-  // stages 2 then 1 per group, activation stages 8 .. 2
+  // stage counts of this list that fit: word stages 2 then 1 per decode
+  // group, activation stages 8 .. 2 (4 groups fit for every code size, N <=
+  // 8192 and NT <= 256: at most 201 KB)
   auto fits = [&](int nt, int sa, int sx, int sw) {
     return (int64_t)gemm_smem(nt, sa, sx, sw, g.BW, d.N).total <= budget;
   };
-  static const int kShapes[][3] = {{4, 8, 8}, {4, 8, 4}, {4, 4, 4}, {4, 8, 2}, {4, 4, 2},
-                                   {2, 4, 4}, {2, 4, 2}, {2, 2, 2}};   // SA, SW, SX
+  static const int kShapes[][3] = {{4, 8, 8}, {4, 8, 4}, {4, 4, 4}, {4, 8, 2}, {4, 4, 2}};   // SA, SW, SX
   int NT = nt_cap(T), SA = 0, SW = 0, SX = 0;
   for (; NT >= 16 && SA == 0; NT -= 16) {
     for (const auto &sh : kShapes) {
