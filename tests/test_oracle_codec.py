@@ -166,6 +166,37 @@ def test_roundtrip_exact_when_codebook_holds_the_points():
     assert np.max(np.abs(What - W) / np.max(np.abs(W), axis=1, keepdims=True)) < 1e-6
 
 
+@pytest.mark.parametrize("seed", [0, 1, 2, 3, 5, 8])
+def test_whole_codec_hand_computed_two_columns(seed):
+    """QAM-W page, Methodology (1)-(6) on one row of two columns, worked by
+    hand: W = (3, 4), s = 1, b = 2, a QPSK codebook (+-1, +-1). r = 5 and
+    u = (0.6, 0.8); y = H_2 (d u) / sqrt 2 is a unit vector, so with one row
+    sigma = sqrt(2/pi) |y| = sqrt(2/pi) and x = y sqrt(pi/2); the nearest
+    centroid is the sign pattern of x; the decode gives
+    w_hat = r d (H_2 sigma c) / sqrt 2. The sign mask d comes from the
+    generator pinned to its published outputs (test_oracle_rotation)."""
+    W = np.array([[3.0, 4.0]], dtype=np.float32)
+    C = np.array([[1, 1], [-1, 1], [-1, -1], [1, -1]], dtype=np.float32)
+    d = codec.sign_mask(seed, 2)
+    y0 = (d[0] * 0.6 + d[1] * 0.8) / math.sqrt(2.0)
+    y1 = (d[0] * 0.6 - d[1] * 0.8) / math.sqrt(2.0)
+    sig_hand = math.sqrt(2.0 / math.pi)
+    sig = codec.calibrate_sigma(W, None, 0.0, 2, seed)
+    assert sig[0] == np.float32(sig_hand)
+    x = np.array([y0, y1]) / float(np.float32(sig_hand))
+    c_hand = (1.0 if x[0] > 0 else -1.0, 1.0 if x[1] > 0 else -1.0)
+    idx_hand = {(1, 1): 0, (-1, 1): 1, (-1, -1): 2, (1, -1): 3}[c_hand]
+    enc = codec.encode(W, None, 0.0, 2, seed, sig, C, 2)
+    assert float(enc["r"][0]) == 5.0
+    assert np.allclose(enc["x"].reshape(-1), x, rtol=1e-6, atol=0)
+    assert int(enc["idx"].reshape(-1)[0]) == idx_hand
+    sg = float(sig[0])
+    yh0, yh1 = sg * c_hand[0], sg * c_hand[1]
+    w_hand = [5.0 * d[0] * (yh0 + yh1) / math.sqrt(2.0), 5.0 * d[1] * (yh0 - yh1) / math.sqrt(2.0)]
+    What = codec.decode(enc["packed"], enc["r"], sig, None, 0.0, 2, 2, seed, C, 2)
+    assert np.allclose(What.reshape(-1), w_hand, rtol=1e-12, atol=1e-12)
+
+
 def test_end_to_end_distortion_matches_codebook_distortion():
     """u unit, K/2 pairs with sigma^2 ~ 1/K: E|u - u_hat|^2 ~ D_B / 2."""
     rng = np.random.default_rng(5)
