@@ -1114,6 +1114,49 @@ def run_decode_gemm(args):
     clk = clocks.stop()
     if status.item() != 0:
         raise SystemExit(f"device status {status.item()} in the timed calls")
+    # end to end at T = 1: the token's activations uploaded from pinned host
+    # memory, the fused call, Y read back, all inside the timed region
+    T1 = DG_TOKENS[0]
+    x_host = Xs[T1].cpu().pin_memory()
+    y_host = torch.empty((T1, M), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(Xs[T1])
+    e2e_ts = []
+    for i in range(args.warmup + max(args.steps, 3)):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        q.decode_matmul(enc, Cd, x_dev, status=status, out=Ys[T1], workspace=Ws[T1])
+        y_host.copy_(Ys[T1], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= args.warmup:
+            e2e_ts.append(e0.elapsed_time(e1))
+    if not torch.equal(y_host, Ys[T1].cpu()):
+        raise SystemExit("end-to-end read-back differs from the device result")
+    e2e_ms = statistics.median(e2e_ts)
+    e2e = {"value": M * K / (e2e_ms * 1e-3) / 1e9, "unit": "Gweights/s",
+           "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+           "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+           "note": "T = 1 token: its activations uploaded, the fused call, Y read back (pinned host memory)"}
+    # the oracle (decode then product, fp64 numpy) on a bounded sample of rows, one core
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0:
+        from oracle import codec as ocodec
+        n_rows = args.cpu_rows or 64
+        idx_o = ocodec.unpack_indices(enc.packed[:n_rows].cpu().numpy().view(np.uint32), K // 2, spec.bits)
+        r_o, sig_o, s_o = enc.row_norm[:n_rows].cpu().numpy(), enc.sigma.cpu().numpy(), enc.col_scale.cpu().numpy()
+        X1 = Xs[T1].double().cpu().numpy()
+        C_o = Cd.cpu().numpy()
+        ts_o = []
+        for _ in range(3):
+            t_a = time.perf_counter()
+            Wh = ocodec.decode_with_scale(idx_o, r_o, sig_o, s_o, K, spec.block, spec.seed, C_o)
+            X1 @ Wh.T
+            ts_o.append(time.perf_counter() - t_a)
+        cpu = {"value": n_rows * K / statistics.median(ts_o) / 1e9, "unit": "Gweights/s", "cores": 1,
+               "kind": "oracle", "sample": f"{n_rows} of {M} rows decoded (fp64) and multiplied with one token; "
+                                           "median of 3"}
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     tc_peak = float(peaks.get("bf16_tflops", 1590.0))
@@ -1145,8 +1188,9 @@ def run_decode_gemm(args):
                     "frac": flops4 / t4 / 1e12 / tc_peak, "traffic": None,
                     "kernel": "prepare_x_kernel + decode_gemm_kernel at T = 4096",
                     "peak_source": f"{peak_kind} bf16_tflops (burst; fp16 runs at the bf16 rate)"}},
-                "per_tokens": rows, "gpu_launches": len(DG_TOKENS) * 3 * max(args.steps, 3),
-                "clocks": clk, "cpu_baseline": None, "e2e": None,
+                "per_tokens": rows,
+                "gpu_launches": len(DG_TOKENS) * 3 * max(args.steps, 3) + 2 * len(e2e_ts),
+                "clocks": clk, "cpu_baseline": cpu, "e2e": e2e,
                 "timing": "each call timed alone with events after an L2 flush; median of the repetitions"}
         print(json.dumps(line), flush=True)
     return 0
