@@ -21,20 +21,25 @@
 //
 // Kernel 2 (decode_gemm_kernel), persistent: one CTA per SM. The work is the
 // list of (output tile, K chunk) units -- an output tile is 128 rows m x NT
-// tokens, a chunk 64 columns (32 pairs) -- split into equal contiguous
-// ranges, one per CTA ("stream-K"), so every SM gets the same number of
-// chunks whatever the number of tiles. Warp roles:
-//   warps 0-15  unpack the chunk's indices of the 128 rows, look the centroids
-//               up as fp16 pairs and write the 128 x 128 operand tile into
-//               shared memory in the tensor cores' swizzled K-major layout;
+// tokens, a chunk 128 columns (64 pairs, two 128-byte swizzle atoms) -- split
+// into equal contiguous ranges, one per CTA ("stream-K"), so every SM gets the
+// same number of chunks whatever the number of tiles. Warp roles:
+//   warps 0-15  two groups of 8; a group unpacks the chunk's indices of the
+//               128 rows (two threads per row, one atom each), looks the
+//               centroids up as fp16 pairs and writes the 128 x 128-column
+//               operand tile into shared memory in the tensor cores' swizzled
+//               K-major layout;
 //   warp 16     streams the packed indices into a ring of word stages (one TMA
 //               tensor copy per chunk, or cp.async when the row pitch is not a
 //               multiple of 16 bytes);
-//   warp 17     streams the fp16 a tile of the chunk (TMA, 128-byte swizzle)
-//               into a ring of its own, running ahead of the operand stages;
-//   warp 18     issues the chunk's four 128 x NT x 16 tcgen05.mma (fp16 in,
+//   warp 17     streams the fp16 a tile of the chunk (two TMA copies, 128-byte
+//               swizzle) into the activation stage beside the group's operand
+//               stage; its bytes complete the same full barrier, so the MMA
+//               warp waits once per chunk;
+//   warp 18     issues the chunk's eight 128 x NT x 16 tcgen05.mma (fp16 in,
 //               fp32 accumulated in tensor memory, two accumulators used in
-//               turn) and commits them to mbarriers;
+//               turn) and commits them to the stage's empty barrier (one
+//               commit frees both tiles);
 //   warps 19-22 read a finished accumulator (tcgen05.ld) and write
 //               Y = r_m 2^e_t acc; a tile whose chunks were split between CTAs
 //               is written as partial sums to the workspace, and the CTA that
@@ -60,14 +65,15 @@ namespace qamw {
 namespace {
 
 constexpr int kBM = 128;                   // output rows per tile (tensor-memory lanes)
-constexpr int kBK = 64;                    // columns (32 pairs) per chunk: one 128-byte swizzle atom
-constexpr int kDecWarps = 16;              // SA groups (4 or 2); a group decodes one unit at a time
+constexpr int kBK = 128;                   // columns (64 pairs) per chunk: two 128-byte swizzle atoms
+constexpr int kAtom = 64;                  // columns of one swizzle atom (128 bytes of fp16)
+constexpr int kDecWarps = 16;              // 2 groups of 8; a group decodes one unit at a time
 constexpr int kWarpWords = kDecWarps;      // streams the packed words
 constexpr int kWarpX = kDecWarps + 1;      // streams the activation tiles
 constexpr int kWarpMma = kDecWarps + 2;    // issues the MMAs
 constexpr int kWarpEpi = kDecWarps + 3;    // first of the 4 epilogue warps
 constexpr int kThreads = (kDecWarps + 7) * 32;
-constexpr int kStageBytesA = kBM * 128;    // the 128-row x 64-column operand tile (one swizzle atom)
+constexpr int kStageBytesA = 2 * kBM * 128;   // the 128-row x 128-column operand tile: [atom][row][128 B]
 constexpr int kMaxStages = 8;
 constexpr int kMaxCtas = 160;              // persistent CTAs at most (the partial-sum slots are sized for it)
 constexpr uint32_t kWaitTries = 1u << 22;  // try_wait attempts before a spinning wait gives up
@@ -106,26 +112,25 @@ struct GemmArgs {
   int64_t n_units;          // tiles x chunks
   int N, bits;
   int NT;                   // tokens per tile (16..256, a multiple of 16)
-  int SA;                   // weight-tile stages = decode groups (4)
+  int SA;                   // weight-tile stages = decode groups (2)
   int SW;                   // word stages (a multiple of SA)
-  int SX;                   // activation-tile stages
   int BW;                   // staged words per row and chunk
   int words_tma;            // 1: words by TMA; 0: by cp.async
   int32_t *status;
 };
 
-// shared-memory layout (after 1024-byte alignment): SA weight tiles, SX
+// shared-memory layout (after 1024-byte alignment): SA weight tiles, SA
 // activation tiles, SW word stages, the fp16 codebook
 struct GemmSmem {
   int stage_x, wpitch;
   size_t off_x, off_w, off_cb, total;
 };
-__host__ __device__ __forceinline__ GemmSmem gemm_smem(int NT, int SA, int SX, int SW, int BW, int N) {
+__host__ __device__ __forceinline__ GemmSmem gemm_smem(int NT, int SA, int SW, int BW, int N) {
   GemmSmem g;
-  g.stage_x = NT * 128;                                  // one atom of NT rows x 128 B
+  g.stage_x = NT * 256;                                  // two atoms of NT rows x 128 B
   g.wpitch = (kBM * BW * 4 + 127) & ~127;
   g.off_x = (size_t)SA * kStageBytesA;
-  g.off_w = g.off_x + (size_t)SX * g.stage_x;
+  g.off_w = g.off_x + (size_t)SA * g.stage_x;
   g.off_cb = g.off_w + (size_t)SW * g.wpitch;
   g.total = g.off_cb + (size_t)N * 4;
   return g;
@@ -252,23 +257,22 @@ struct Cursor {
   }
 };
 
-// The operand row of one unit: the 32 fp16 centroid pairs of row rl, written
-// in the 128-byte swizzled K-major layout (pairs 16 j .. 16 j + 15 = 16-byte
-// chunks 4 j .. 4 j + 3; chunk position XOR rl % 8, so the 8 rows of a
-// quarter-warp hit 8 different bank groups). Field k of the row's chunk is
-// bits 32 REM + k BB .. of the staged words w. Returns the status bits.
+// One atom of an operand row: the 32 fp16 centroid pairs of row rl in one
+// 64-column half of the unit, written in the 128-byte swizzled K-major layout
+// (pairs 16 j .. 16 j + 15 = 16-byte chunks 4 j .. 4 j + 3; chunk position XOR
+// rl % 8, so the 8 rows of a quarter-warp hit 8 different bank groups). Field
+// k of the half is bits 32 REM + k BB .. of the staged words w. Returns the
+// status bits.
 template <int BB>
 struct RowWords {
   static constexpr int kNW4 = (96 + 32 * BB + 127) / 128;   // 16-byte loads that cover REM <= 3 plus 32 fields
 };
 template <int BB, int REM>
 __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<BB>::kNW4], const uint32_t *cb,
-                                              unsigned char *arow, int rl, int jb, int nb, bool check_idx, int N,
-                                              bool rin) {
+                                              unsigned char *arow, int rl, bool check_idx, int N, bool rin) {
   uint32_t bad = 0;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    if (j < jb || j >= jb + nb) continue;   // the batches of this thread's part of the row
     uint32_t e[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
@@ -291,10 +295,9 @@ __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<B
 }
 // the same for a code size known only at run time (fields read from shared memory)
 __device__ __forceinline__ uint32_t write_row_any(const uint32_t *rowp, int rem, int B, const uint32_t *cb,
-                                                  unsigned char *arow, int rl, int jb, int nb, bool check_idx,
-                                                  int N, bool rin) {
+                                                  unsigned char *arow, int rl, bool check_idx, int N, bool rin) {
   uint32_t bad = 0;
-  for (int j = jb; j < jb + nb; ++j) {
+  for (int j = 0; j < 2; ++j) {
     uint32_t e[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
@@ -523,15 +526,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 1024-byte alignment for the swizzled operand tiles
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int B = BB > 0 ? BB : g.bits;
-  const int NT = g.NT, SA = g.SA, SW = g.SW, SX = g.SX;
-  const GemmSmem L = gemm_smem(NT, SA, SX, SW, g.BW, g.N);
+  const int NT = g.NT, SA = g.SA, SW = g.SW;
+  const GemmSmem L = gemm_smem(NT, SA, SW, g.BW, g.N);
   unsigned char *A0 = smem;                                          // [SA][kStageBytesA]
-  unsigned char *X0 = smem + L.off_x;                                // [SX][stage_x]
+  unsigned char *X0 = smem + L.off_x;                                // [SA][stage_x]
   unsigned char *W0 = smem + L.off_w;                                // [SW][wpitch]
   uint32_t *cb = reinterpret_cast<uint32_t *>(smem + L.off_cb);      // [N] fp16 pairs
 
   __shared__ __align__(8) uint64_t full_w[kMaxStages], empty_w[kMaxStages];
-  __shared__ __align__(8) uint64_t full_x[kMaxStages], empty_x[kMaxStages], full_a[kMaxStages], empty_a[kMaxStages];
+  __shared__ __align__(8) uint64_t full_a[kMaxStages], empty_a[kMaxStages];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
@@ -555,12 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty_w[s], kDecWarps / SA);   // the warps of the group that decodes the stage's units
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(&full_a[s], kDecWarps / SA);
+      mbar_init(&full_a[s], kDecWarps / SA + 1);   // the group's warps + the activation warp (with its bytes)
       mbar_init(&empty_a[s], 1);
-    }
-    for (int s = 0; s < SX; ++s) {
-      mbar_init(&full_x[s], 1);
-      mbar_init(&empty_x[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&acc_full[s], 1);
@@ -583,21 +582,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool failed = false;
 
   if (warp < kDecWarps) {
-    // ---- decode: SA groups of 16 / SA warps; group grp takes the CTA's units
+    // ---- decode: SA = 2 groups of 8 warps; group grp takes the CTA's units
     // u0 + grp, u0 + grp + SA, ... into operand stage grp and word stages
     // grp, grp + SA, ... (each stage is used by one group, in order), so SA
     // units are decoded at once. In a unit, thread tg of the group owns row
-    // rl = tg % 128 and batches jb .. jb + nb - 1 of its 2 batches of 16 pairs.
+    // rl = tg % 128 and half hf = tg / 128 of it: the 32 pairs of atom hf,
+    // whose B words start hf B words after the unit's first word.
     const int wpg = kDecWarps / SA;
     const int grp = warp / wpg;
     const int tg = (warp % wpg) * 32 + lane;
     const int rl = tg & (kBM - 1);
-    const int nb = SA / 2;             // batches per thread: 2 (SA = 4, one thread per row) or 1 (two)
-    const int jb = (tg >> 7) * nb;
+    const int hf = tg >> 7;
     const bool check_idx = g.N < (1 << B);
     int sw = grp;
     uint32_t qa = 0, qw = 0;   // stage use counts (phase = count & 1)
-    unsigned char *arow = A0 + (size_t)grp * kStageBytesA + rl * 128;
+    unsigned char *arow = A0 + (size_t)grp * kStageBytesA + (size_t)hf * (kBM * 128) + rl * 128;
     Cursor cur(u0 + grp, n_chunks, g.n_m);
     for (int64_t u = u0 + grp; u < u1; u += SA) {
       const int c = cur.c;
@@ -605,8 +604,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every failure decision is taken by the whole warp (the loop holds warp-wide syncs)
       int r = wait_phase(&full_w[sw], qw & 1u, fail);
       if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
-      const int rem = g.words_tma ? ((c * B) & 3) : 0;   // the chunk's first word in the staged row
-      const uint32_t *rowp = reinterpret_cast<const uint32_t *>(W0 + (size_t)sw * L.wpitch) + rl * g.BW;
+      // the half's first word in the staged row: the unit's 2B words start 0..3
+      // words into it (TMA) or at its start (cp.async)
+      const int s0 = (g.words_tma ? ((c * 2 * B) & 3) : 0) + hf * B;
+      const int rem = s0 & 3;
+      const uint32_t *rowp = reinterpret_cast<const uint32_t *>(W0 + (size_t)sw * L.wpitch) + rl * g.BW + (s0 & ~3);
       if (BB > 0) {
         constexpr int kNW4 = RowWords<BB>::kNW4;
         uint32_t w[4 * kNW4];
@@ -626,17 +628,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
         }
         switch (rem) {
-          case 0: bad |= write_row<BB, 0>(w, cb, arow, rl, jb, nb, check_idx, g.N, rin); break;
-          case 1: bad |= write_row<BB, 1>(w, cb, arow, rl, jb, nb, check_idx, g.N, rin); break;
-          case 2: bad |= write_row<BB, 2>(w, cb, arow, rl, jb, nb, check_idx, g.N, rin); break;
-          default: bad |= write_row<BB, 3>(w, cb, arow, rl, jb, nb, check_idx, g.N, rin); break;
+          case 0: bad |= write_row<BB, 0>(w, cb, arow, rl, check_idx, g.N, rin); break;
+          case 1: bad |= write_row<BB, 1>(w, cb, arow, rl, check_idx, g.N, rin); break;
+          case 2: bad |= write_row<BB, 2>(w, cb, arow, rl, check_idx, g.N, rin); break;
+          default: bad |= write_row<BB, 3>(w, cb, arow, rl, check_idx, g.N, rin); break;
         }
       } else {
         if (qa > 0) {
           r = wait_phase(&empty_a[grp], (qa & 1u) ^ 1u, fail);
           if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
         }
-        bad |= write_row_any(rowp, rem, B, cb, arow, rl, jb, nb, check_idx, g.N, rin);
+        bad |= write_row_any(rowp, rem, B, cb, arow, rl, check_idx, g.N, rin);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_w[sw]);
       }
@@ -665,17 +667,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g.words_tma) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&full_w[sw], (uint32_t)(kBM * g.BW * 4));
-          tma_load_2d(dst, &wmap, (c * B) & ~3, (int)m0, &full_w[sw]);
+          tma_load_2d(dst, &wmap, (c * 2 * B) & ~3, (int)m0, &full_w[sw]);
         }
       } else {
-        // a row's B words of the chunk, 4 bytes at a time; rows past M are
-        // not copied (their stale words decode to in-range centroids of rows
-        // that are never written)
+        // a row's 2B words of the chunk, 4 bytes at a time; rows past M are
+        // not copied (their stale words decode to centroids of rows that are
+        // never written)
         for (int row = lane; row < kBM; row += 32) {
           if (m0 + row < g.M) {
-            const uint32_t *src = g.packed + (m0 + row) * g.wpr + (int64_t)c * B;
+            const uint32_t *src = g.packed + (m0 + row) * g.wpr + (int64_t)c * 2 * B;
             uint32_t *d = reinterpret_cast<uint32_t *>(dst) + row * g.BW;
-            for (int k = 0; k < B; ++k) cp_async4(d + k, src + k);
+            for (int k = 0; k < 2 * B; ++k) cp_async4(d + k, src + k);
           }
         }
         cp_async_arrive_noinc(&full_w[sw]);
@@ -693,7 +695,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kWarpX) {
-    // ---- activation tile of each unit -> activation stage (u - u0) % SX
+    // ---- activation tile of each unit -> activation stage (u - u0) % SA, the
+    // one beside the unit's operand stage: its copies complete on the same
+    // full barrier as the decode group's tile (one wait for the MMA warp), and
+    // the stage is free again when that tile's MMAs are (empty_a)
     if (lane == 0) {
       int sx = 0;
       uint32_t px = 0;
@@ -703,27 +708,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t u = u0; u < u1; ++u, cur.next(n_chunks, g.n_m)) {
         const int c = cur.c;
         const int64_t t0 = cur.tt * NT;
-        if (u - u0 >= SX) {
-          const int r = wait_phase(&empty_x[sx], px ^ 1u, fail);
+        if (u - u0 >= SA) {
+          const int r = wait_phase(&empty_a[sx], px ^ 1u, fail);
           if (r) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
         }
         unsigned char *dst = X0 + (size_t)sx * L.stage_x;
-        mbar_arrive_expect_tx(&full_x[sx], (uint32_t)L.stage_x);
-        tma_load_2d(dst, &xmap, c * kBK, (int)t0, &full_x[sx]);
+        mbar_arrive_expect_tx(&full_a[sx], (uint32_t)L.stage_x);
+        tma_load_2d(dst, &xmap, c * kBK, (int)t0, &full_a[sx]);                   // atom 0: NT x 64 columns
+        tma_load_2d(dst + NT * 128, &xmap, c * kBK + kAtom, (int)t0, &full_a[sx]);  // atom 1
         issued = u - u0 + 1;
-        if (++sx == SX) { sx = 0; px ^= 1u; }
+        if (++sx == SA) { sx = 0; px ^= 1u; }
       }
+      // copies still in flight land before the CTA exits (bounded: the phase
+      // also waits for the decode group, which may have stopped)
       if (failed)
-        for (int64_t i = (issued > SX ? issued - SX : 0); i < issued; ++i)
-          mbar_wait(&full_x[i % SX], (uint32_t)((i / SX) & 1), kWaitTries);
+        for (int64_t i = (issued > SA ? issued - SA : 0); i < issued; ++i)
+          mbar_wait(&full_a[i % SA], (uint32_t)((i / SA) & 1), kWaitTries);
     }
   } else if (warp == kWarpMma) {
     // ---- MMA issue; segment = the CTA's units of one tile, accumulated in buffer seg % 2
     if (lane == 0) {
       // instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = NT, M = 128
       const uint32_t idesc = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-      int sa = 0, sx = 0;
-      uint32_t pa = 0, px = 0;
+      int sa = 0;
+      uint32_t pa = 0;
       int64_t seg = 0;
       bool any = false;
       int c = (int)(u0 % n_chunks);
@@ -733,29 +741,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t buf = (uint32_t)(seg & 1);
         int r = 0;
         if (first && seg >= 2) r = wait_phase(&acc_empty[buf], (uint32_t)(((seg >> 1) - 1) & 1), fail);
-        if (!r) r = wait_phase(&full_a[sa], pa, fail);
-        if (!r) r = wait_phase(&full_x[sx], px, fail);
+        if (!r) r = wait_phase(&full_a[sa], pa, fail);   // the operand tile and the activation tile
         if (r) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(A0 + (size_t)sa * kStageBytesA);
-        const uint32_t b_base = smem_u32(X0 + (size_t)sx * L.stage_x);
+        // descriptors of the stage's first atoms; a step along K adds its byte
+        // offset / 16 to the start-address field (no carry: shared-memory
+        // addresses stay below 2^18)
+        const uint64_t ad0 = smem_desc_sw128(smem_u32(A0 + (size_t)sa * kStageBytesA));
+        const uint64_t bd0 = smem_desc_sw128(smem_u32(X0 + (size_t)sa * L.stage_x));
         const uint32_t d = tmem + buf * acc_cols;
 #pragma unroll
         for (int k16 = 0; k16 < kBK / 16; ++k16) {
-          const uint32_t koff = k16 * 32;   // 16 columns = 32 bytes along the swizzled row
-          const uint64_t ad = smem_desc_sw128(a_base + koff);
-          const uint64_t bd = smem_desc_sw128(b_base + koff);
+          // atom k16 / 4 (16 KB apart in A, NT x 128 B in the activations);
+          // 16 columns = 32 bytes along its swizzled rows
+          const uint64_t ad = ad0 + (uint64_t)((k16 >> 2) * (kBM * 128 / 16) + (k16 & 3) * 2);
+          const uint64_t bd = bd0 + (uint64_t)((k16 >> 2) * (NT * 128 / 16) + (k16 & 3) * 2);
           mma_f16(d, ad, bd, idesc, (!first || k16 > 0) ? 1u : 0u);
         }
-        mma_commit(&empty_a[sa]);
-        mma_commit(&empty_x[sx]);
+        mma_commit(&empty_a[sa]);   // frees the operand stage and the activation stage
         any = true;
         if (last) {
           mma_commit(&acc_full[buf]);
           ++seg;
         }
         if (++sa == SA) { sa = 0; pa ^= 1u; }
-        if (++sx == SX) { sx = 0; px ^= 1u; }
       }
       if (any) {   // every MMA issued completes before the tensor memory is freed
         const int ls = (sa + SA - 1) % SA;                  // stage of the last committed unit
@@ -894,11 +903,12 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   g.status = d.status;
   const int B = d.bits;
   // the packed words by TMA when the row pitch is a multiple of 16 bytes: a
-  // chunk's B words start at word Bc, 0 to 3 words past a 16-byte boundary,
-  // so a box of B + 3 words (rounded up to 4) holds them; cp.async copies
-  // place them at the start of the staged row
+  // chunk's 2B words start at word 2Bc, 0 to 3 words past a 16-byte boundary;
+  // cp.async copies place them at the start of the staged row. The thread of
+  // the second half reads 16-byte groups from the one holding word B + 3 at
+  // most, enough of them to cover 3 + B words: the row holds both reads.
   g.words_tma = ((d.wpr * 4) % 16 == 0 && reinterpret_cast<uintptr_t>(d.packed) % 16 == 0) ? 1 : 0;
-  g.BW = (B + 3 + 3) & ~3;
+  g.BW = ((B + 3) & ~3) + ((B + 3 + 3) & ~3);
   if ((g.BW / 4) % 2 == 0) g.BW += 4;   // an odd number of 16-byte groups per row: rows hit different banks
   // kernel 1's CTA shape: a cluster of up to 8 CTAs per token for few tokens
   // (its latency is on the critical path), one CTA per token from 512 tokens
@@ -910,31 +920,26 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   const int prep_S = T >= 512 ? 1 : (int)std::min<int64_t>(kPrepCluster, prep_units);
   const size_t prep_smem = (size_t)((prep_units + prep_S - 1) / prep_S) * ucols * 4;
   const int64_t budget = (int64_t)smem_max - 1024 - 256 - (prep_S > 1 ? (int64_t)prep_smem + 2048 : 0);
-  // the widest token tile (<= 256, a multiple of 16) and, for it, the first
-  // stage counts of this list that fit: word stages 2 then 1 per decode
-  // group, activation stages 8 .. 2 (4 groups fit for every code size, N <=
-  // 8192 and NT <= 256: at most 201 KB)
-  auto fits = [&](int nt, int sa, int sx, int sw) {
-    return (int64_t)gemm_smem(nt, sa, sx, sw, g.BW, d.N).total <= budget;
-  };
-  static const int kShapes[][3] = {{4, 8, 8}, {4, 8, 4}, {4, 4, 4}, {4, 8, 2}, {4, 4, 2}};   // SA, SW, SX
-  int NT = nt_cap(T), SA = 0, SW = 0, SX = 0;
-  for (; NT >= 16 && SA == 0; NT -= 16) {
-    for (const auto &sh : kShapes) {
-      if (fits(NT, sh[0], sh[2], sh[1])) {
-        SA = sh[0];
-        SW = sh[1];
-        SX = sh[2];
+  // two decode groups, each with its operand and activation stage; the
+  // widest token tile (<= 256, a multiple of 16) and, for it, the most word
+  // stages per group (4, 2, 1) that fit (the smallest shape fits every code
+  // size and N <= 8192 at NT = 16: at most 140 KB)
+  const int SA = 2;
+  auto fits = [&](int nt, int sw) { return (int64_t)gemm_smem(nt, SA, sw, g.BW, d.N).total <= budget; };
+  int NT = nt_cap(T), SW = 0;
+  for (; NT >= 16 && SW == 0; NT -= 16) {
+    for (const int sw : {4 * SA, 2 * SA, SA}) {
+      if (fits(NT, sw)) {
+        SW = sw;
         break;
       }
     }
-    if (SA != 0) break;
+    if (SW != 0) break;
   }
-  if (SA == 0) return cudaErrorNotSupported;
+  if (SW == 0) return cudaErrorNotSupported;
   g.NT = NT;
   g.SA = SA;
   g.SW = SW;
-  g.SX = SX;
   g.n_m = (d.M + kBM - 1) / kBM;
   const int64_t n_tiles = g.n_m * ((T + NT - 1) / NT);
   g.n_units = n_tiles * (d.K / kBK);
@@ -977,7 +982,7 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   {
     cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)T};
     cuuint64_t strides[1] = {(cuuint64_t)d.K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)NT};
+    cuuint32_t box[2] = {(cuuint32_t)kAtom, (cuuint32_t)NT};
     cuuint32_t es[2] = {1, 1};
     if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, A, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -996,7 +1001,7 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   } else {
     wmap = xmap;   // unused
   }
-  const size_t smem = 1024 + gemm_smem(NT, SA, SX, SW, g.BW, d.N).total;
+  const size_t smem = 1024 + gemm_smem(NT, SA, SW, g.BW, d.N).total;
   auto run = [&](auto kern) -> cudaError_t {
     cudaError_t err = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
     if (err != cudaSuccess) return err;
