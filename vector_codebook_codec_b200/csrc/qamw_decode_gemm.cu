@@ -153,6 +153,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.p
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }   // the 4 epilogue warps
+__device__ __forceinline__ void dec_sync() { asm volatile("bar.sync 2, 512;" ::: "memory"); }   // the 16 decode warps
 // barrier of the 4 epilogue warps that returns whether any of their threads passed true
 __device__ __forceinline__ bool epi_any(bool v) {
   uint32_t r;
@@ -548,10 +549,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t acc_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
   const uint32_t tmem_cols = 2 * acc_cols;
 
-  for (int i = threadIdx.x; i < g.N; i += kThreads) {
-    const __half2 h = __floats2half2_rn(g.codebook[2 * i], g.codebook[2 * i + 1]);
-    cb[i] = *reinterpret_cast<const uint32_t *>(&h);
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW; ++s) {
       mbar_init(&full_w[s], g.words_tma ? 1 : 32);
@@ -582,6 +579,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool failed = false;
 
   if (warp < kDecWarps) {
+    // the fp16 codebook, filled by the decode warps alone while the copy
+    // warps already start streaming the first stages
+    for (int i = threadIdx.x; i < g.N; i += kDecWarps * 32) {
+      const __half2 h = __floats2half2_rn(g.codebook[2 * i], g.codebook[2 * i + 1]);
+      cb[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    dec_sync();
     // ---- decode: SA = 2 groups of 8 warps; group grp takes the CTA's units
     // u0 + grp, u0 + grp + SA, ... into operand stage grp and word stages
     // grp, grp + SA, ... (each stage is used by one group, in order), so SA
