@@ -21,25 +21,28 @@
 //
 // Kernel 2 (decode_gemm_kernel), persistent: one CTA per SM. The work is the
 // list of (output tile, K chunk) units -- an output tile is 128 rows m x NT
-// tokens, a chunk 128 columns (64 pairs, two 128-byte swizzle atoms) -- split
-// into equal contiguous ranges, one per CTA ("stream-K"), so every SM gets the
-// same number of chunks whatever the number of tiles. Warp roles:
+// tokens, a chunk 128 columns (64 pairs) -- split into equal contiguous
+// ranges, one per CTA ("stream-K"), so every SM gets the same number of
+// chunks whatever the number of tiles. Warp roles:
 //   warps 0-15  two groups of 8; a group unpacks the chunk's indices of the
-//               128 rows (two threads per row, one atom each), looks the
-//               centroids up as fp16 pairs and writes the 128 x 128-column
-//               operand tile into shared memory in the tensor cores' swizzled
-//               K-major layout;
+//               128 rows (two threads per row, one 64-column half each), looks
+//               the centroids up as fp16 pairs and stores the 128 x 128-column
+//               operand tile straight into tensor memory (tcgen05.st: row m in
+//               lane m, pair k in column k), where the MMA reads it -- the
+//               decoded weights never touch shared memory;
 //   warp 16     streams the packed indices into a ring of word stages (one TMA
 //               tensor copy per chunk, or cp.async when the row pitch is not a
 //               multiple of 16 bytes);
 //   warp 17     streams the fp16 a tile of the chunk (two TMA copies, 128-byte
-//               swizzle) into the activation stage beside the group's operand
-//               stage; its bytes complete the same full barrier, so the MMA
-//               warp waits once per chunk;
-//   warp 18     issues the chunk's eight 128 x NT x 16 tcgen05.mma (fp16 in,
-//               fp32 accumulated in tensor memory, two accumulators used in
-//               turn) and commits them to the stage's empty barrier (one
-//               commit frees both tiles);
+//               swizzle, two atoms of 64 columns) into the shared-memory
+//               activation stage that goes with the group's operand stage; its
+//               bytes complete the same full barrier, so the MMA warp waits
+//               once per chunk;
+//   warp 18     issues the chunk's eight 128 x NT x 16 tcgen05.mma (A from
+//               tensor memory, B from shared memory, fp16 in, fp32 accumulated
+//               in tensor memory, two accumulators used in turn for NT <= 128)
+//               and commits them to the stage's empty barrier (one commit
+//               frees both tiles);
 //   warps 19-22 read a finished accumulator (tcgen05.ld) and write
 //               Y = r_m 2^e_t acc; a tile whose chunks were split between CTAs
 //               is written as partial sums to the workspace, and the CTA that
@@ -73,7 +76,6 @@ constexpr int kWarpX = kDecWarps + 1;      // streams the activation tiles
 constexpr int kWarpMma = kDecWarps + 2;    // issues the MMAs
 constexpr int kWarpEpi = kDecWarps + 3;    // first of the 4 epilogue warps
 constexpr int kThreads = (kDecWarps + 7) * 32;
-constexpr int kStageBytesA = 2 * kBM * 128;   // the 128-row x 128-column operand tile: [atom][row][128 B]
 constexpr int kMaxStages = 8;
 constexpr int kMaxCtas = 160;              // persistent CTAs at most (the partial-sum slots are sized for it)
 constexpr uint32_t kWaitTries = 1u << 22;  // try_wait attempts before a spinning wait gives up
@@ -119,8 +121,8 @@ struct GemmArgs {
   int32_t *status;
 };
 
-// shared-memory layout (after 1024-byte alignment): SA weight tiles, SA
-// activation tiles, SW word stages, the fp16 codebook
+// shared-memory layout (after 1024-byte alignment): SA activation tiles, SW
+// word stages, the fp16 codebook (the operand tiles live in tensor memory)
 struct GemmSmem {
   int stage_x, wpitch;
   size_t off_x, off_w, off_cb, total;
@@ -129,7 +131,7 @@ __host__ __device__ __forceinline__ GemmSmem gemm_smem(int NT, int SA, int SW, i
   GemmSmem g;
   g.stage_x = NT * 256;                                  // two atoms of NT rows x 128 B
   g.wpitch = (kBM * BW * 4 + 127) & ~127;
-  g.off_x = (size_t)SA * kStageBytesA;
+  g.off_x = 0;
   g.off_w = g.off_x + (size_t)SA * g.stage_x;
   g.off_cb = g.off_w + (size_t)SW * g.wpitch;
   g.total = g.off_cb + (size_t)N * 4;
@@ -149,7 +151,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }   // the 4 epilogue warps
@@ -185,15 +186,24 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -258,19 +268,19 @@ struct Cursor {
   }
 };
 
-// One atom of an operand row: the 32 fp16 centroid pairs of row rl in one
-// 64-column half of the unit, written in the 128-byte swizzled K-major layout
-// (pairs 16 j .. 16 j + 15 = 16-byte chunks 4 j .. 4 j + 3; chunk position XOR
-// rl % 8, so the 8 rows of a quarter-warp hit 8 different bank groups). Field
-// k of the half is bits 32 REM + k BB .. of the staged words w. Returns the
-// status bits.
+// One half of an operand row: the 32 fp16 centroid pairs of one 64-column
+// half of the unit, stored into tensor-memory columns ta .. ta + 31 of the
+// thread's lane (pair k in column k: the K-major layout of an A operand read
+// from tensor memory, two fp16 per 32-bit column). Field k of the half is bits
+// 32 REM + k BB .. of the staged words w. Warp-collective (tcgen05.st); returns
+// the status bits.
 template <int BB>
 struct RowWords {
   static constexpr int kNW4 = (96 + 32 * BB + 127) / 128;   // 16-byte loads that cover REM <= 3 plus 32 fields
 };
 template <int BB, int REM>
 __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<BB>::kNW4], const uint32_t *cb,
-                                              unsigned char *arow, int rl, bool check_idx, int N, bool rin) {
+                                              uint32_t ta, bool check_idx, int N, bool rin) {
   uint32_t bad = 0;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
@@ -287,16 +297,13 @@ __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<B
       }
       e[p] = cb[id];
     }
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch)
-      *reinterpret_cast<uint4 *>(arow + (((4 * j + ch) ^ (rl & 7)) << 4)) =
-          make_uint4(e[4 * ch], e[4 * ch + 1], e[4 * ch + 2], e[4 * ch + 3]);
+    tmem_st16(ta + 16 * j, e);   // pairs 16 j .. 16 j + 15 = tensor-memory columns
   }
   return bad;
 }
 // the same for a code size known only at run time (fields read from shared memory)
 __device__ __forceinline__ uint32_t write_row_any(const uint32_t *rowp, int rem, int B, const uint32_t *cb,
-                                                  unsigned char *arow, int rl, bool check_idx, int N, bool rin) {
+                                                  uint32_t ta, bool check_idx, int N, bool rin) {
   uint32_t bad = 0;
   for (int j = 0; j < 2; ++j) {
     uint32_t e[16];
@@ -312,10 +319,7 @@ __device__ __forceinline__ uint32_t write_row_any(const uint32_t *rowp, int rem,
       }
       e[p] = cb[id];
     }
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch)
-      *reinterpret_cast<uint4 *>(arow + (((4 * j + ch) ^ (rl & 7)) << 4)) =
-          make_uint4(e[4 * ch], e[4 * ch + 1], e[4 * ch + 2], e[4 * ch + 3]);
+    tmem_st16(ta + 16 * j, e);
   }
   return bad;
 }
@@ -529,7 +533,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B = BB > 0 ? BB : g.bits;
   const int NT = g.NT, SA = g.SA, SW = g.SW;
   const GemmSmem L = gemm_smem(NT, SA, SW, g.BW, g.N);
-  unsigned char *A0 = smem;                                          // [SA][kStageBytesA]
   unsigned char *X0 = smem + L.off_x;                                // [SA][stage_x]
   unsigned char *W0 = smem + L.off_w;                                // [SW][wpitch]
   uint32_t *cb = reinterpret_cast<uint32_t *>(smem + L.off_cb);      // [N] fp16 pairs
@@ -546,8 +549,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_chunks = (int)(g.K / kBK);
   const int64_t G = gridDim.x;
   const int64_t u0 = range_start(blockIdx.x, G, g.n_units), u1 = range_start(blockIdx.x + 1, G, g.n_units);
+  // tensor memory: nbuf accumulators of acc_cols columns (two, so that the
+  // epilogue of one tile overlaps the MMAs of the next, unless NT > 128),
+  // then the SA operand stages of 64 columns (128 fp16 per lane)
   const uint32_t acc_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
-  const uint32_t tmem_cols = 2 * acc_cols;
+  const uint32_t lbuf = 2 * acc_cols + 64 * SA <= 512 ? 1 : 0;   // log2 of the accumulator count
+  const uint32_t nbuf = 1u << lbuf;
+  const uint32_t a_col0 = nbuf * acc_cols;
+  const uint32_t tmem_cols = a_col0 + 64 * SA <= 256 ? 256 : 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW; ++s) {
@@ -590,8 +599,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // u0 + grp, u0 + grp + SA, ... into operand stage grp and word stages
     // grp, grp + SA, ... (each stage is used by one group, in order), so SA
     // units are decoded at once. In a unit, thread tg of the group owns row
-    // rl = tg % 128 and half hf = tg / 128 of it: the 32 pairs of atom hf,
-    // whose B words start hf B words after the unit's first word.
+    // rl = tg % 128 and half hf = tg / 128 of it: the 32 pairs of columns
+    // 64 hf .. 64 hf + 63, whose B words start hf B words after the unit's
+    // first word. Row rl is tensor-memory lane rl (32 (warp % 4) + lane, the
+    // lanes this warp may access); stage grp's half hf is columns
+    // a_col0 + 64 grp + 32 hf .. + 31.
     const int wpg = kDecWarps / SA;
     const int grp = warp / wpg;
     const int tg = (warp % wpg) * 32 + lane;
@@ -600,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool check_idx = g.N < (1 << B);
     int sw = grp;
     uint32_t qa = 0, qw = 0;   // stage use counts (phase = count & 1)
-    unsigned char *arow = A0 + (size_t)grp * kStageBytesA + (size_t)hf * (kBM * 128) + rl * 128;
+    const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + a_col0 + 64 * grp + 32 * hf;
     Cursor cur(u0 + grp, n_chunks, g.n_m);
     for (int64_t u = u0 + grp; u < u1; u += SA) {
       const int c = cur.c;
@@ -630,23 +642,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (qa > 0) {   // the stage's previous MMAs are done with it
           r = wait_phase(&empty_a[grp], (qa & 1u) ^ 1u, fail);
           if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+          tc_fence_after();
         }
         switch (rem) {
-          case 0: bad |= write_row<BB, 0>(w, cb, arow, rl, check_idx, g.N, rin); break;
-          case 1: bad |= write_row<BB, 1>(w, cb, arow, rl, check_idx, g.N, rin); break;
-          case 2: bad |= write_row<BB, 2>(w, cb, arow, rl, check_idx, g.N, rin); break;
-          default: bad |= write_row<BB, 3>(w, cb, arow, rl, check_idx, g.N, rin); break;
+          case 0: bad |= write_row<BB, 0>(w, cb, ta, check_idx, g.N, rin); break;
+          case 1: bad |= write_row<BB, 1>(w, cb, ta, check_idx, g.N, rin); break;
+          case 2: bad |= write_row<BB, 2>(w, cb, ta, check_idx, g.N, rin); break;
+          default: bad |= write_row<BB, 3>(w, cb, ta, check_idx, g.N, rin); break;
         }
       } else {
         if (qa > 0) {
           r = wait_phase(&empty_a[grp], (qa & 1u) ^ 1u, fail);
           if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
+          tc_fence_after();
         }
-        bad |= write_row_any(rowp, rem, B, cb, arow, rl, check_idx, g.N, rin);
+        bad |= write_row_any(rowp, rem, B, cb, ta, check_idx, g.N, rin);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_w[sw]);
       }
-      fence_proxy_async_smem();   // the tile's generic stores become visible to the tensor cores
+      tmem_st_wait();   // the tile's tensor-memory stores are done
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_a[grp]);
       for (int k = 0; k < SA; ++k) cur.next(n_chunks, g.n_m);
@@ -730,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&full_a[i % SA], (uint32_t)((i / SA) & 1), kWaitTries);
     }
   } else if (warp == kWarpMma) {
-    // ---- MMA issue; segment = the CTA's units of one tile, accumulated in buffer seg % 2
+    // ---- MMA issue; segment = the CTA's units of one tile, accumulated in buffer seg % nbuf
     if (lane == 0) {
       // instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = NT, M = 128
       const uint32_t idesc = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
@@ -742,25 +757,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t u = u0; u < u1; ++u, c = (c + 1 == n_chunks) ? 0 : c + 1) {
         const bool first = (u == u0) || (c == 0);
         const bool last = (u + 1 == u1) || (c == n_chunks - 1);
-        const uint32_t buf = (uint32_t)(seg & 1);
+        const uint32_t buf = (uint32_t)seg & (nbuf - 1);
         int r = 0;
-        if (first && seg >= 2) r = wait_phase(&acc_empty[buf], (uint32_t)(((seg >> 1) - 1) & 1), fail);
+        if (first && seg >= nbuf) r = wait_phase(&acc_empty[buf], (uint32_t)(((seg >> lbuf) - 1) & 1), fail);
         if (!r) r = wait_phase(&full_a[sa], pa, fail);   // the operand tile and the activation tile
         if (r) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
         tc_fence_after();
         // descriptors of the stage's first atoms; a step along K adds its byte
         // offset / 16 to the start-address field (no carry: shared-memory
         // addresses stay below 2^18)
-        const uint64_t ad0 = smem_desc_sw128(smem_u32(A0 + (size_t)sa * kStageBytesA));
+        const uint32_t ta0 = tmem + a_col0 + 64 * sa;
         const uint64_t bd0 = smem_desc_sw128(smem_u32(X0 + (size_t)sa * L.stage_x));
         const uint32_t d = tmem + buf * acc_cols;
 #pragma unroll
         for (int k16 = 0; k16 < kBK / 16; ++k16) {
           // atom k16 / 4 (16 KB apart in A, NT x 128 B in the activations);
           // 16 columns = 32 bytes along its swizzled rows
-          const uint64_t ad = ad0 + (uint64_t)((k16 >> 2) * (kBM * 128 / 16) + (k16 & 3) * 2);
           const uint64_t bd = bd0 + (uint64_t)((k16 >> 2) * (NT * 128 / 16) + (k16 & 3) * 2);
-          mma_f16(d, ad, bd, idesc, (!first || k16 > 0) ? 1u : 0u);
+          mma_f16_ts(d, ta0 + 8 * k16, bd, idesc, (!first || k16 > 0) ? 1u : 0u);   // 16 columns of A = 8 tensor-memory columns
         }
         mma_commit(&empty_a[sa]);   // frees the operand stage and the activation stage
         any = true;
@@ -786,9 +800,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tile = u / n_chunks, c_begin = u - tile * n_chunks;
       const int64_t seg_end = (u1 < (tile + 1) * n_chunks) ? u1 : (tile + 1) * n_chunks;
       const bool whole = c_begin == 0 && seg_end == (tile + 1) * n_chunks;
-      const uint32_t buf = (uint32_t)(seg & 1);
+      const uint32_t buf = (uint32_t)seg & (nbuf - 1);
       // one decision for all 4 warps: the partial-sum path below holds their named barriers
-      const int r = wait_phase_sleep(&acc_full[buf], (uint32_t)((seg >> 1) & 1), fail);
+      const int r = wait_phase_sleep(&acc_full[buf], (uint32_t)((seg >> lbuf) & 1), fail);
       if (epi_any(r != 0)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
       tc_fence_after();
       const int64_t tt = tile / g.n_m;
@@ -924,10 +938,11 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   const int prep_S = T >= 512 ? 1 : (int)std::min<int64_t>(kPrepCluster, prep_units);
   const size_t prep_smem = (size_t)((prep_units + prep_S - 1) / prep_S) * ucols * 4;
   const int64_t budget = (int64_t)smem_max - 1024 - 256 - (prep_S > 1 ? (int64_t)prep_smem + 2048 : 0);
-  // two decode groups, each with its operand and activation stage; the
-  // widest token tile (<= 256, a multiple of 16) and, for it, the most word
-  // stages per group (4, 2, 1) that fit (the smallest shape fits every code
-  // size and N <= 8192 at NT = 16: at most 140 KB)
+  // two decode groups, each with its operand stage (tensor memory) and
+  // activation stage (shared memory); the widest token tile (<= 256, a
+  // multiple of 16) and, for it, the most word stages per group (4, 2, 1)
+  // that fit (the smallest shape fits every code size and N <= 8192 at
+  // NT = 16: at most 76 KB)
   const int SA = 2;
   auto fits = [&](int nt, int sw) { return (int64_t)gemm_smem(nt, SA, sw, g.BW, d.N).total <= budget; };
   int NT = nt_cap(T), SW = 0;
