@@ -165,6 +165,12 @@ __device__ __forceinline__ bool epi_any(bool v) {
   return r != 0;
 }
 
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -558,6 +564,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t a_col0 = nbuf * acc_cols;
   const uint32_t tmem_cols = a_col0 + 64 * SA <= 256 ? 256 : 512;
 
+  // each decode thread requests its first 4 codebook entries before the setup,
+  // so that their latency overlaps it (and comes before the copies' burst)
+  constexpr int kCbPre = 4;
+  const bool cb_vec = (reinterpret_cast<uintptr_t>(g.codebook) & 7) == 0;
+  float2 cpre[kCbPre];
+#pragma unroll
+  for (int k = 0; k < kCbPre; ++k) {
+    const int i = threadIdx.x + k * kDecWarps * 32;
+    cpre[k] = (warp < kDecWarps && cb_vec && i < g.N) ? reinterpret_cast<const float2 *>(g.codebook)[i]
+                                                       : make_float2(0.0f, 0.0f);
+  }
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < SW; ++s) {
       mbar_init(&full_w[s], g.words_tma ? 1 : 32);
@@ -590,9 +608,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kDecWarps) {
     // the fp16 codebook, filled by the decode warps alone while the copy
     // warps already start streaming the first stages
-    for (int i = threadIdx.x; i < g.N; i += kDecWarps * 32) {
-      const __half2 h = __floats2half2_rn(g.codebook[2 * i], g.codebook[2 * i + 1]);
-      cb[i] = *reinterpret_cast<const uint32_t *>(&h);
+    if (cb_vec) {   // 8-byte loads: the first kCbPre per thread already in registers
+#pragma unroll
+      for (int k = 0; k < kCbPre; ++k) {
+        const int i = threadIdx.x + k * kDecWarps * 32;
+        const __half2 h = __floats2half2_rn(cpre[k].x, cpre[k].y);
+        if (i < g.N) cb[i] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+#pragma unroll 4
+      for (int i = threadIdx.x + kCbPre * kDecWarps * 32; i < g.N; i += kDecWarps * 32) {
+        const float2 c2 = reinterpret_cast<const float2 *>(g.codebook)[i];
+        const __half2 h = __floats2half2_rn(c2.x, c2.y);
+        cb[i] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+    } else {
+      for (int i = threadIdx.x; i < g.N; i += kDecWarps * 32) {
+        const __half2 h = __floats2half2_rn(g.codebook[2 * i], g.codebook[2 * i + 1]);
+        cb[i] = *reinterpret_cast<const uint32_t *>(&h);
+      }
     }
     dec_sync();
     // ---- decode: SA = 2 groups of 8 warps; group grp takes the CTA's units
@@ -841,12 +874,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
         const int64_t b_first = cta_of_unit(tile * n_chunks, G, g.n_units);
         const int64_t b_last = cta_of_unit((tile + 1) * n_chunks - 1, G, g.n_units);
-        __threadfence();
-        epi_sync();
+        epi_sync();   // the 4 warps' partial sums are written
         if (threadIdx.x == kWarpEpi * 32) {
-          const uint32_t old = atomicAdd(&g.counters[tile], 1u);
+          // release: this CTA's partial sums (ordered before it by the barrier)
+          // are visible with its count; acquire: the last contributor sees all
+          // the others' (and passes them on to its warps through the barrier)
+          const uint32_t old = atom_add_acq_rel(&g.counters[tile], 1u);
           s_last = (old == (uint32_t)(b_last - b_first)) ? 1 : 0;
-          __threadfence();
         }
         epi_sync();
         if (s_last) {
@@ -964,39 +998,8 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
   g.n_units = n_tiles * (d.K / kBK);
   const int64_t G = std::min<int64_t>(std::min<int64_t>(sm_count(), kMaxCtas), g.n_units);
 
-  // ---- kernel 1: a cluster of S CTAs per token
-  {
-    PrepArgs p;
-    p.X = X;
-    p.ldx = ldx;
-    p.T = T;
-    p.K = d.K;
-    p.sigma = d.sigma;
-    p.col_scale = d.col_scale;
-    p.seed = d.seed;
-    p.log2b = d.log2b;
-    p.A = A;
-    p.tok_scale = tok_scale;
-    p.counters = counters;
-    p.n_counters = n_tiles;
-    p.S = prep_S;
-    const size_t smem = prep_smem;
-    if ((e = set_max_dynamic_smem(reinterpret_cast<const void *>(prepare_x_kernel), smem)) != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.S * T), 1, 1);
-    cfg.blockDim = dim3(kPrepThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if ((e = cudaLaunchKernelEx(&cfg, prepare_x_kernel, p)) != cudaSuccess) return e;
-  }
-
+  // everything on the host first (tensor maps, attributes), so that the two
+  // launches follow each other at once: kernel 2 starts beside kernel 1
   CUtensorMap xmap, wmap;
   {
     cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)T};
@@ -1021,9 +1024,47 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
     wmap = xmap;   // unused
   }
   const size_t smem = 1024 + gemm_smem(NT, SA, SW, g.BW, d.N).total;
+  // 11- and 10-bit codes compiled for their shape; anything else at run time
+  const void *kfn = B == 11   ? reinterpret_cast<const void *>(decode_gemm_kernel<11>)
+                    : B == 10 ? reinterpret_cast<const void *>(decode_gemm_kernel<10>)
+                              : reinterpret_cast<const void *>(decode_gemm_kernel<0>);
+  if ((e = set_max_dynamic_smem(kfn, smem)) != cudaSuccess) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void *>(prepare_x_kernel), prep_smem)) != cudaSuccess) return e;
+
+  // ---- kernel 1: a cluster of S CTAs per token
+  {
+    PrepArgs p;
+    p.X = X;
+    p.ldx = ldx;
+    p.T = T;
+    p.K = d.K;
+    p.sigma = d.sigma;
+    p.col_scale = d.col_scale;
+    p.seed = d.seed;
+    p.log2b = d.log2b;
+    p.A = A;
+    p.tok_scale = tok_scale;
+    p.counters = counters;
+    p.n_counters = n_tiles;
+    p.S = prep_S;
+    const size_t smem = prep_smem;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.S * T), 1, 1);
+    cfg.blockDim = dim3(kPrepThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, prepare_x_kernel, p)) != cudaSuccess) return e;
+  }
+
+
   auto run = [&](auto kern) -> cudaError_t {
-    cudaError_t err = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
-    if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1036,7 +1077,6 @@ cudaError_t launch_decode_gemm(const DecodeArgs &d, const uint16_t *X, int64_t T
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, xmap, wmap, g);
   };
-  // 11- and 10-bit codes compiled for their shape; anything else at run time
   if (B == 11) return run(decode_gemm_kernel<11>);
   if (B == 10) return run(decode_gemm_kernel<10>);
   return run(decode_gemm_kernel<0>);
