@@ -284,9 +284,10 @@ template <int BB>
 struct RowWords {
   static constexpr int kNW4 = (96 + 32 * BB + 127) / 128;   // 16-byte loads that cover REM <= 3 plus 32 fields
 };
-template <int BB, int REM>
+// CHECK: the codebook has fewer than 2^B entries, so a field may be out of range.
+template <int BB, int REM, bool CHECK>
 __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<BB>::kNW4], const uint32_t *cb,
-                                              uint32_t ta, bool check_idx, int N, bool rin) {
+                                              uint32_t ta, int N, bool rin) {
   uint32_t bad = 0;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
@@ -294,10 +295,10 @@ __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<B
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
       const int b = 32 * REM + (16 * j + p) * BB, wi = b >> 5, sh = b & 31;
-      uint32_t v = w[wi] >> sh;
-      if (sh + BB > 32) v |= w[wi + 1] << (32 - sh);
+      // one funnel shift for a field that spans two words
+      const uint32_t v = (sh + BB > 32) ? __funnelshift_r(w[wi], w[wi + 1], sh) : (w[wi] >> sh);
       uint32_t id = v & ((1u << BB) - 1u);
-      if (check_idx && id >= (uint32_t)N) {   // a codebook smaller than 2^B: decode as centroid 0
+      if (CHECK && id >= (uint32_t)N) {   // decode as centroid 0
         if (rin) bad |= QAMW_STATUS_BAD_INDEX;
         id = 0;
       }
@@ -677,11 +678,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (__reduce_max_sync(0xffffffffu, (unsigned)r)) { if (r == 2) bad |= QAMW_STATUS_TIMEOUT; failed = true; break; }
           tc_fence_after();
         }
-        switch (rem) {
-          case 0: bad |= write_row<BB, 0>(w, cb, ta, check_idx, g.N, rin); break;
-          case 1: bad |= write_row<BB, 1>(w, cb, ta, check_idx, g.N, rin); break;
-          case 2: bad |= write_row<BB, 2>(w, cb, ta, check_idx, g.N, rin); break;
-          default: bad |= write_row<BB, 3>(w, cb, ta, check_idx, g.N, rin); break;
+        if (check_idx) {
+          switch (rem) {
+            case 0: bad |= write_row<BB, 0, true>(w, cb, ta, g.N, rin); break;
+            case 1: bad |= write_row<BB, 1, true>(w, cb, ta, g.N, rin); break;
+            case 2: bad |= write_row<BB, 2, true>(w, cb, ta, g.N, rin); break;
+            default: bad |= write_row<BB, 3, true>(w, cb, ta, g.N, rin); break;
+          }
+        } else {
+          switch (rem) {
+            case 0: write_row<BB, 0, false>(w, cb, ta, g.N, rin); break;
+            case 1: write_row<BB, 1, false>(w, cb, ta, g.N, rin); break;
+            case 2: write_row<BB, 2, false>(w, cb, ta, g.N, rin); break;
+            default: write_row<BB, 3, false>(w, cb, ta, g.N, rin); break;
+          }
         }
       } else {
         if (qa > 0) {
