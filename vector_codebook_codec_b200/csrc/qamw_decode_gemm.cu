@@ -288,6 +288,8 @@ struct RowWords {
 template <int BB, int REM, bool CHECK>
 __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<BB>::kNW4], const uint32_t *cb,
                                               uint32_t ta, int N, bool rin) {
+  constexpr uint32_t kMask4 = ((1u << BB) - 1u) << 2;   // the field times 4: its byte offset in the table
+  const unsigned char *cbb = reinterpret_cast<const unsigned char *>(cb);
   uint32_t bad = 0;
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
@@ -295,14 +297,16 @@ __device__ __forceinline__ uint32_t write_row(const uint32_t (&w)[4 * RowWords<B
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
       const int b = 32 * REM + (16 * j + p) * BB, wi = b >> 5, sh = b & 31;
-      // one funnel shift for a field that spans two words
-      const uint32_t v = (sh + BB > 32) ? __funnelshift_r(w[wi], w[wi + 1], sh) : (w[wi] >> sh);
-      uint32_t id = v & ((1u << BB) - 1u);
-      if (CHECK && id >= (uint32_t)N) {   // decode as centroid 0
+      // the byte offset 4 id straight from the words: one shift (a funnel
+      // shift for a field that spans two words) and one mask
+      uint32_t off = (sh + BB > 32) ? (__funnelshift_r(w[wi], w[wi + 1], sh - 2) & kMask4)
+                     : (sh >= 2)    ? ((w[wi] >> (sh - 2)) & kMask4)
+                                    : ((w[wi] << (2 - sh)) & kMask4);
+      if (CHECK && off >= ((uint32_t)N << 2)) {   // decode as centroid 0
         if (rin) bad |= QAMW_STATUS_BAD_INDEX;
-        id = 0;
+        off = 0;
       }
-      e[p] = cb[id];
+      e[p] = *reinterpret_cast<const uint32_t *>(cbb + off);
     }
     tmem_st16(ta + 16 * j, e);   // pairs 16 j .. 16 j + 15 = tensor-memory columns
   }
