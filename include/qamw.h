@@ -337,9 +337,10 @@ int qamw_decode(const uint32_t *packed, const float *row_norm, const float *sigm
  * A first kernel computes a_t in fp32 and stores it in the workspace as fp16,
  * scaled by a power of two 2^-e_t per token (its largest |a| lands in
  * (2^13, 2^14]); a second streams the packed indices, looks up the centroids
- * as fp16 pairs into the tensor-core operand tile in shared memory, multiplies
- * on the tensor cores (tcgen05, fp32 accumulation in tensor memory) and
- * scales by r_m 2^e_t. The weights never reach device memory.
+ * as fp16 pairs and stores them straight into the tensor-core A operand in
+ * tensor memory, multiplies on the tensor cores (tcgen05, fp32 accumulation in
+ * tensor memory) and scales by r_m 2^e_t. The weights never reach device
+ * memory, nor shared memory.
  * Accuracy: with S[t][m] = r_m sum_i |a_t[i] C[idx(m,i/2)][i%2]| and
  * Q[t][m] = r_m sum_i sigma_{i/2} |C[..]| sum_{j in block(i)} |X[t][j] / s_j| / sqrt(b),
  *   |Y - Y_exact| <= (2^-10 + K 2^-22) S + 2^-19 Q + (tiny fp16-subnormal terms),
