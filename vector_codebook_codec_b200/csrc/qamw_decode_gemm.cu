@@ -75,7 +75,8 @@ constexpr int kWarpWords = kDecWarps;      // streams the packed words
 constexpr int kWarpX = kDecWarps + 1;      // streams the activation tiles
 constexpr int kWarpMma = kDecWarps + 2;    // issues the MMAs
 constexpr int kWarpEpi = kDecWarps + 3;    // first of the 4 epilogue warps
-constexpr int kThreads = (kDecWarps + 7) * 32;
+constexpr int kWarpMma2 = kDecWarps + 7;   // the second MMA issuer for token tiles of <= 64
+constexpr int kThreads = (kDecWarps + 8) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kMaxCtas = 160;              // persistent CTAs at most (the partial-sum slots are sized for it)
 constexpr uint32_t kWaitTries = 1u << 22;  // try_wait attempts before a spinning wait gives up
@@ -227,6 +228,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 accumulator columns of this warp's lanes: the sum of the ni accumulators
+// (acc_cols apart) that the MMA warps filled
+__device__ __forceinline__ void tmem_ld_acc(uint32_t taddr, uint32_t ni, uint32_t acc_cols, float (&v)[16]) {
+  tmem_ld16(taddr, v);
+  if (ni == 2) {
+    float v2[16];
+    tmem_ld16(taddr + acc_cols, v2);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += v2[j];
+  }
 }
 
 // Bounded waits that also give up once another role of the CTA has failed:
@@ -560,13 +573,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_chunks = (int)(g.K / kBK);
   const int64_t G = gridDim.x;
   const int64_t u0 = range_start(blockIdx.x, G, g.n_units), u1 = range_start(blockIdx.x + 1, G, g.n_units);
-  // tensor memory: nbuf accumulators of acc_cols columns (two, so that the
-  // epilogue of one tile overlaps the MMAs of the next, unless NT > 128),
+  // tensor memory: nbuf accumulator buffers (two, so that the epilogue of one
+  // tile overlaps the MMAs of the next, unless NT > 128), each of ni
+  // accumulators of acc_cols columns (two for NT <= 64: the two MMA warps
+  // each sum one 64-column half of every unit, and the epilogue adds them),
   // then the SA operand stages of 64 columns (128 fp16 per lane)
   const uint32_t acc_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
-  const uint32_t lbuf = 2 * acc_cols + 64 * SA <= 512 ? 1 : 0;   // log2 of the accumulator count
+  const uint32_t ni = NT <= 64 ? 2 : 1;
+  const uint32_t lbuf = 2 * ni * acc_cols + 64 * SA <= 512 ? 1 : 0;   // log2 of the buffer count
   const uint32_t nbuf = 1u << lbuf;
-  const uint32_t a_col0 = nbuf * acc_cols;
+  const uint32_t a_col0 = nbuf * ni * acc_cols;
   const uint32_t tmem_cols = a_col0 + 64 * SA <= 256 ? 256 : 512;
 
   // each decode thread requests its first 4 codebook entries before the setup,
@@ -588,10 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(&full_a[s], kDecWarps / SA + 1);   // the group's warps + the activation warp (with its bytes)
-      mbar_init(&empty_a[s], 1);
+      mbar_init(&empty_a[s], ni);   // a commit of each MMA warp
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_full[s], ni);
       mbar_init(&acc_empty[s], 4);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -791,9 +807,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int64_t i = (issued > SA ? issued - SA : 0); i < issued; ++i)
           mbar_wait(&full_a[i % SA], (uint32_t)((i / SA) & 1), kWaitTries);
     }
-  } else if (warp == kWarpMma) {
-    // ---- MMA issue; segment = the CTA's units of one tile, accumulated in buffer seg % nbuf
-    if (lane == 0) {
+  } else if (warp == kWarpMma || warp == kWarpMma2) {
+    // ---- MMA issue; segment = the CTA's units of one tile, accumulated in
+    // buffer seg % nbuf. With ni = 2 MMA warp mi issues the 4 MMAs of atom mi
+    // of every unit into accumulator mi: two issuers halve the serial chain of
+    // one thread (each of its tensor and shared-memory instructions queues
+    // behind the decode warps' gathers)
+    const int mi = warp == kWarpMma ? 0 : 1;
+    if (lane == 0 && mi < (int)ni) {
       // instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, N = NT, M = 128
       const uint32_t idesc = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
       int sa = 0;
@@ -815,13 +836,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // addresses stay below 2^18)
         const uint32_t ta0 = tmem + a_col0 + 64 * sa;
         const uint64_t bd0 = smem_desc_sw128(smem_u32(X0 + (size_t)sa * L.stage_x));
-        const uint32_t d = tmem + buf * acc_cols;
+        const uint32_t d = tmem + (buf * ni + mi) * acc_cols;
+        const int kb = 4 * mi, nk = (kBK / 16) / ni;   // this warp's K steps: kb .. kb + nk - 1
 #pragma unroll
-        for (int k16 = 0; k16 < kBK / 16; ++k16) {
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          if (kk >= nk) break;
+          const int k16 = kb + kk;
           // atom k16 / 4 (16 KB apart in A, NT x 128 B in the activations);
           // 16 columns = 32 bytes along its swizzled rows
           const uint64_t bd = bd0 + (uint64_t)((k16 >> 2) * (NT * 128 / 16) + (k16 & 3) * 2);
-          mma_f16_ts(d, ta0 + 8 * k16, bd, idesc, (!first || k16 > 0) ? 1u : 0u);   // 16 columns of A = 8 tensor-memory columns
+          mma_f16_ts(d, ta0 + 8 * k16, bd, idesc, (!first || kk > 0) ? 1u : 0u);   // 16 columns of A = 8 tensor-memory columns
         }
         mma_commit(&empty_a[sa]);   // frees the operand stage and the activation stage
         any = true;
@@ -857,11 +881,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t t0 = tt * NT;
       const float rn = m < g.M ? g.row_norm[m] : 0.0f;
       if (m < g.M && !isfinite(rn)) bad |= QAMW_STATUS_NONFINITE_NORM;
-      const uint32_t taddr = tmem + buf * acc_cols + ((uint32_t)(32 * wq) << 16);
+      const uint32_t taddr = tmem + buf * ni * acc_cols + ((uint32_t)(32 * wq) << 16);
       if (whole) {
         for (int c0 = 0; c0 < NT; c0 += 16) {
           float v[16];
-          tmem_ld16(taddr + (uint32_t)c0, v);
+          tmem_ld_acc(taddr + (uint32_t)c0, ni, acc_cols, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int64_t t = t0 + c0 + j;
@@ -879,7 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float *mine = g.part + ((size_t)(2 * blockIdx.x + slot) * NT) * kBM;
         for (int c0 = 0; c0 < NT; c0 += 16) {
           float v[16];
-          tmem_ld16(taddr + (uint32_t)c0, v);
+          tmem_ld_acc(taddr + (uint32_t)c0, ni, acc_cols, v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) mine[(size_t)(c0 + j) * kBM + row] = v[j];
         }
