@@ -927,8 +927,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
             for (int64_t b = b_first; b <= b_last; ++b) {
-              // CTA b holds this tile in its first segment unless its range began in an earlier tile
-              const int sl = (range_start(b, G, g.n_units) < tile * n_chunks) ? 1 : 0;
+              // CTA b holds this tile in its first segment unless its range
+              // began in an earlier tile (only b_first can have)
+              const int sl = (b == b_first && range_start(b, G, g.n_units) < tile * n_chunks) ? 1 : 0;
               const float *pp = g.part + ((size_t)(2 * b + sl) * NT) * kBM;
 #pragma unroll
               for (int j = 0; j < 16; ++j) acc[j] += __ldcg(pp + (size_t)(c0 + j) * kBM + row);
