@@ -108,6 +108,7 @@ def _check(M, K, T, block, N, bits, seed, with_scale=True):
 @pytest.mark.parametrize("M,K,T,block,N,bits", [
     (128, 128, 16, 128, 2048, 11),      # one tile, one chunk; 88-byte rows: words by cp.async
     (256, 512, 40, 128, 2048, 11),      # two row tiles, four chunks (TMA words), a partial token tile (40 of 48)
+    (256, 1024, 100, 128, 2048, 11),    # a 112-token tile: one MMA warp, two accumulators of 128 columns
     (200, 256, 1, 64, 256, 8),          # ragged rows (TMA zero fill), one token, b = 64
     (200, 384, 5, 128, 2048, 11),       # ragged rows with the cp.async words (3 x 88-byte chunks per row)
     (128, 384, 256, 32, 1024, 10),      # a full 256-token tile, b = 32
@@ -200,3 +201,20 @@ def test_fused_decode_matmul_reuses_a_caller_workspace():
     Y1 = qamw.decode_matmul(enc, Cd, X, workspace=ws)
     Y2 = qamw.decode_matmul(enc, Cd, X, workspace=ws)
     assert torch.equal(Y0, Y1) and torch.equal(Y1, Y2)
+
+
+def test_fused_decode_matmul_codebook_at_a_4_byte_offset():
+    """A codebook that starts 4 bytes past an 8-byte boundary: the kernel fills
+    its table with 4-byte loads instead of the 8-byte ones (same values)."""
+    M, K, T, block, N, bits, seed = 256, 512, 16, 128, 2048, 11, 27
+    enc, Cd, Xb, *_ = _case(M, K, T, block, N, bits, seed)
+    buf = torch.zeros(2 * N + 1, dtype=torch.float32, device="cuda")
+    buf[1:] = Cd.reshape(-1)
+    C_off = buf[1:].view(N, 2)
+    assert C_off.data_ptr() % 8 == 4
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y_aligned = qamw.decode_matmul(enc, Cd, Xb.cuda(), status=st)
+    Y_off = qamw.decode_matmul(enc, C_off, Xb.cuda(), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(Y_aligned, Y_off)
