@@ -39,10 +39,11 @@
 //               bytes complete the same full barrier, so the MMA warp waits
 //               once per chunk;
 //   warp 18     issues the chunk's eight 128 x NT x 16 tcgen05.mma (A from
-//               tensor memory, B from shared memory, fp16 in, fp32 accumulated
-//               in tensor memory, two accumulators used in turn for NT <= 128)
-//               and commits them to the stage's empty barrier (one commit
-//               frees both tiles);
+//   (and 23)    tensor memory, B from shared memory, fp16 in, fp32 accumulated
+//               in tensor memory, two accumulator buffers used in turn for
+//               NT <= 128) and commits them to the stage's empty barrier (that
+//               commit frees both tiles); for NT <= 64 warp 23 issues the four
+//               of the chunk's second atom into an accumulator of its own;
 //   warps 19-22 read a finished accumulator (tcgen05.ld) and write
 //               Y = r_m 2^e_t acc; a tile whose chunks were split between CTAs
 //               is written as partial sums to the workspace, and the CTA that
@@ -384,7 +385,10 @@ __device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t ran
   return v;
 }
 
-// at most 48 registers: one CTA fits beside a CTA of kernel 2 (736 threads x 80 registers)
+// 48 registers, no spills. A CTA does not fit beside a CTA of kernel 2 (24
+// warps x 80 registers leave 1024 registers per SM sub-partition): kernel 2's
+// CTAs on the few SMs that run kernel 1 start when it ends. A 32-register
+// build that fits beside it was measured no faster (its spills).
 __global__ void __launch_bounds__(kPrepThreads, 10) prepare_x_kernel(PrepArgs p) {
   extern __shared__ __align__(16) float vloc[];   // the CTA's units, fp32, one after the other
   __shared__ float red[kPrepThreads / 32];
