@@ -231,6 +231,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // 16 accumulator columns of this warp's lanes: the sum of the ni accumulators
 // (acc_cols apart) that the MMA warps filled
 __device__ __forceinline__ void tmem_ld_acc(uint32_t taddr, uint32_t ni, uint32_t acc_cols, float (&v)[16]) {
@@ -911,9 +921,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) mine[(size_t)(c0 + j) * kBM + row] = v[j];
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        // with two accumulator buffers this one stays held until the part sum
+        // below, which then reads this CTA's own part from tensor memory
+        // instead of back from the workspace (the same values); with one, the
+        // next tile's MMAs need it at once
+        const bool hold = nbuf == 2;
+        if (!hold) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
         const int64_t b_first = cta_of_unit(tile * n_chunks, G, g.n_units);
         const int64_t b_last = cta_of_unit((tile + 1) * n_chunks - 1, G, g.n_units);
         epi_sync();   // the 4 warps' partial sums are written
@@ -931,6 +948,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
             for (int64_t b = b_first; b <= b_last; ++b) {
+              if (hold && b == (int64_t)blockIdx.x) {   // 8 columns at a time: few live registers
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  float v[8];
+                  tmem_ld8(taddr + (uint32_t)(c0 + 8 * h), v);
+                  if (ni == 2) {
+                    float v2[8];
+                    tmem_ld8(taddr + acc_cols + (uint32_t)(c0 + 8 * h), v2);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] += v2[j];
+                  }
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) acc[8 * h + j] += v[j];
+                }
+                continue;
+              }
               // CTA b holds this tile in its first segment unless its range
               // began in an earlier tile (only b_first can have)
               const int sl = (b == b_first && range_start(b, G, g.n_units) < tile * n_chunks) ? 1 : 0;
@@ -944,6 +977,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (m < g.M && t < g.T) g.Y[t * g.ldy + m] = (acc[j] * rn) * g.tok_scale[t];
             }
           }
+        }
+        if (hold) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
         epi_sync();   // s_last is read by all before the next part overwrites it
       }
