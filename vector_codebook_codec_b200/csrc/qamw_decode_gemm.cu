@@ -47,7 +47,8 @@
 //   warps 19-22 read a finished accumulator (tcgen05.ld) and write
 //               Y = r_m 2^e_t acc; a tile whose chunks were split between CTAs
 //               is written as partial sums to the workspace, and the CTA that
-//               finishes it last adds the parts in a fixed order.
+//               finishes it last adds the parts in a fixed order (its own
+//               from its accumulator when there are two).
 // Stages hand over through mbarriers (full / empty per stage), so the roles
 // run ahead of one another by up to the ring depth; no CTA-wide barrier sits
 // in the loop.
